@@ -1,0 +1,37 @@
+"""CPU oracle for tile-routed FP16/INT8 causal prefill attention (TileMix).
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import, call,
+link or run anything in this package.  The library's product path never does:
+it fails loudly when its CUDA extension is missing instead of falling back here.
+
+The oracle is plain and slow on purpose: numpy for block quantisation
+(``quant.py``), pure Python for the routing templates (``routing.py``, with its
+own splitmix64), and plain C in fp64 / int64 for the attention rows
+(``attention_oracle.c``, OpenMP over rows, no blocking).  It shares no code,
+header, table or constant generator with the CUDA path.
+
+Pages followed: "TileMix: Tile-Centric Mixed-Precision Attention for LLM
+Inference Acceleration" (agihunt.info summary, method paragraphs), "Precision
+Has a Map: TileMix Routes INT8 Inside Dense Attention" (cognaptus.com, sections
+"Dense attention does not require uniform precision" and "The routing mechanism
+is designed to stay inside the hot loop"), and the 59188saintaubert.com
+explainer (steps one to three).
+
+Pins: every function here is checked by ``tests/test_oracle_pins.py`` against
+brute force, closed forms, hand-derived words and invariants the pages fix.
+The fp16 output values themselves have no printed worked example on the pages:
+beyond those invariants, output-value parity is unpinned.
+"""
+from .attention import all_rows, attention_rows, build, half_to_double, int_scores
+from .quant import quantize_blocks, quantize_k, quantize_q
+from .routing import (BLOCK_M, BLOCK_N, MAX_GROUPS, TEMPLATES, auto_g, build_routing,
+                      fp16_groups, int8_target, last_legal_tile, legal_groups, n_ktiles,
+                      n_qtiles, tile_offsets)
+
+__all__ = [
+    "BLOCK_M", "BLOCK_N", "MAX_GROUPS", "TEMPLATES", "all_rows", "attention_rows", "auto_g",
+    "build", "build_routing", "fp16_groups", "half_to_double", "int8_target", "int_scores",
+    "last_legal_tile", "legal_groups", "n_ktiles", "n_qtiles", "quantize_blocks",
+    "quantize_k", "quantize_q", "tile_offsets",
+]

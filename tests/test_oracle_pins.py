@@ -1,0 +1,421 @@
+"""Pins of the CPU oracle against brute force, closed forms, hand-derived
+words and the invariants the TileMix pages state.  CPU only."""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import bruteforce as bf
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [x.strip() for x in f if x.strip() and not x.startswith("#")]
+
+
+def _inputs(lengths, hq, hk, d, seed=0):
+    T = sum(lengths)
+    q, k, v = synth.make_qkv(seed, T, hq, hk, d)
+    q8, qs = oracle.quantize_q(q, lengths)
+    k8, ks = oracle.quantize_k(k, lengths)
+    return q, k, v, q8, qs, k8, ks
+
+
+def _words(lengths, hk, value):
+    tm = sum(oracle.n_qtiles(L) for L in lengths)
+    return np.full((tm, hk), value, dtype=np.uint64)
+
+
+def _run(inp, masks, g, lengths, causal, kv_map=None, scale=None):
+    q, k, v, q8, qs, k8, ks = inp
+    O, lse = oracle.attention_rows(q, k, v, q8, qs, k8, ks, masks, g, lengths, causal,
+                                   kv_map=kv_map, scale=scale)
+    T, hq, d = q.shape
+    rows = oracle.all_rows(lengths, hq)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    full = np.zeros((T, hq, d))
+    full_lse = np.zeros((hq, T))
+    t = cu[rows[:, 0]] + rows[:, 2]
+    full[t, rows[:, 1]] = O
+    full_lse[rows[:, 1], t] = lse
+    return full, full_lse
+
+
+# --------------------------------------------------------------------------
+# generator pins
+# --------------------------------------------------------------------------
+
+def test_splitmix64_reference_outputs():
+    want = [int(x, 16) for x in _golden_lines("splitmix64_state0.txt")]
+    assert [synth.draw(0, k) for k in (1, 2, 3)] == want
+    assert [oracle.routing._draw(0, k) for k in (1, 2, 3)] == want
+    lib = synth._load()
+    assert [lib.synth_draw(0, k) for k in (1, 2, 3)] == want
+
+
+def test_box_muller_moments():
+    x = synth.normals(123, 1, 1 << 20)
+    assert abs(x.mean()) < 5e-3
+    assert abs(x.std() - 1.0) < 5e-3
+    # fourth moment of N(0,1) is 3
+    assert abs((x ** 4).mean() - 3.0) < 0.05
+    # any window equals the same slice of a longer draw
+    assert np.array_equal(synth.normals(123, 1, 77, start=1001), x[1001:1078])
+
+
+def test_half_to_double_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits])
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all()
+
+
+# --------------------------------------------------------------------------
+# quantiser pins
+# --------------------------------------------------------------------------
+
+def test_quantiser_hand_cases():
+    for line in _golden_lines("quant_hand_cases.txt"):
+        vals, codes = line.split(";")
+        vals = np.array([float(x) for x in vals.split()], dtype=np.float64)
+        codes = np.array([int(x) for x in codes.split()], dtype=np.int64)
+        x = np.zeros((64, 1, vals.size), dtype=np.float16)
+        x[0, 0] = vals
+        x[1, 0, 0] = 127.0   # absmax of the block is 127 -> scale 1
+        c, s = oracle.quantize_k(x, [64])
+        assert s[0, 0] == np.float32(1.0)
+        assert np.array_equal(c[0, 0].astype(np.int64), codes)
+
+
+def test_quantiser_zero_block_and_tails():
+    # zero block: scale 0, codes 0
+    x = np.zeros((64, 2, 8), dtype=np.float16)
+    x[:, 1] = 1.0
+    c, s = oracle.quantize_k(x, [64])
+    assert s[0, 0] == 0 and not c[:, 0].any()
+    assert s[1, 0] == np.float32(1.0) / np.float32(127.0) and (c[:, 1] == 127).all()
+    # tail block of a 100-row sequence uses rows 64..99 only; a second
+    # sequence's rows never enter the first sequence's blocks
+    lengths = [100, 50]
+    x = np.zeros((150, 1, 4), dtype=np.float16)
+    x[:64] = 1.0
+    x[64:100] = 0.5
+    x[99, 0, 3] = -2.0     # absmax of seq 0 block 1 sits in its last row
+    x[100, 0, 0] = 1000.0  # first row of seq 1
+    c, s = oracle.quantize_k(x, lengths)
+    assert s.shape == (1, 2 + 1)
+    assert s[0, 1] == np.float32(2.0) / np.float32(127.0)
+    assert c[99, 0, 3] == -127 and c[64, 0, 0] == round(0.5 / float(s[0, 1]))
+    assert s[0, 2] == np.float32(1000.0) / np.float32(127.0)
+    # Q blocks are 128 rows
+    cq, sq = oracle.quantize_q(x, lengths)
+    assert sq.shape == (1, 1 + 1)
+    assert sq[0, 0] == np.float32(2.0) / np.float32(127.0)
+
+
+def test_quantiser_error_bound_random():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((300, 3, 64)) * rng.uniform(0.01, 50, (1, 3, 1))).astype(np.float16)
+    lengths = [130, 170]
+    for block, fn in ((64, oracle.quantize_k), (128, oracle.quantize_q)):
+        c, s = fn(x, lengths)
+        t0, col = 0, 0
+        for L in lengths:
+            nb = -(-L // block)
+            for b in range(nb):
+                r0, r1 = t0 + b * block, min(t0 + L, t0 + (b + 1) * block)
+                for h in range(3):
+                    blk = x[r0:r1, h].astype(np.float64)
+                    cc = c[r0:r1, h].astype(np.float64)
+                    sc = float(s[h, col + b])
+                    assert np.abs(cc).max() == 127
+                    assert np.all(np.abs(cc) <= 127)
+                    # |code * s - x| <= s / 2 up to fp32 rounding of x / s
+                    assert np.all(np.abs(cc * sc - blk) <= sc * (0.5 + 1e-5))
+            t0 += L
+            col += nb
+
+
+# --------------------------------------------------------------------------
+# routing pins
+# --------------------------------------------------------------------------
+
+def test_geometry_closed_forms():
+    # L = 4096, g = 1: row qt has 2qt + 2 legal groups, N = 1056 per sequence
+    assert [oracle.legal_groups(qt, 4096, 1, True) for qt in (0, 1, 31)] == [2, 4, 64]
+    assert sum(oracle.legal_groups(qt, 4096, 1, True) for qt in range(32)) == 1056
+    # L = 8192, g = 2: n = qt + 1, N = 2080;  L = 65536, g = 16: N = 16640
+    assert sum(oracle.legal_groups(qt, 8192, 2, True) for qt in range(64)) == 2080
+    assert sum(oracle.legal_groups(qt, 65536, 16, True) for qt in range(512)) == 16640
+    # ragged: L = 100 -> one q-tile, key tiles 0..1
+    assert oracle.last_legal_tile(0, 100, True) == 1
+    assert oracle.last_legal_tile(0, 100, False) == 1
+    assert [oracle.auto_g(L) for L in (64, 4096, 4097, 8192, 65536, 16384)] == [1, 1, 2, 2, 16, 4]
+    cu_q, cu_k = oracle.tile_offsets([100, 256, 64])
+    assert list(cu_q) == [0, 1, 3, 4] and list(cu_k) == [0, 2, 6, 7]
+
+
+def test_band_tiny_golden():
+    want = [int(x, 16) for x in _golden_lines("band_tiny_l256.txt")]
+    m, legal, int8 = oracle.build_routing("band", 50, 0, [256], 1, [1], True)
+    assert [int(x) for x in m[:, 0]] == want
+    assert list(legal) == [6] and list(int8) == [3]
+
+
+def _workload_geometry(name):
+    w = synth.WORKLOADS[name]
+    lengths = synth.workload_lengths(name)
+    if w["g"] == "auto":
+        g = [oracle.auto_g(L) for L in lengths]
+    else:
+        g = [int(w["g"])] * len(lengths)
+    return lengths, g, w
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+@pytest.mark.parametrize("template", oracle.TEMPLATES)
+def test_coverage_exact(name, template):
+    lengths, g, w = _workload_geometry(name)
+    for p in (0, 25, 50, 75, 100):
+        m, legal, int8 = oracle.build_routing(template, p, 3, lengths, 2, g, w["causal"])
+        row = 0
+        for s, L in enumerate(lengths):
+            n = [oracle.legal_groups(qt, L, g[s], w["causal"]) for qt in range(oracle.n_qtiles(L))]
+            assert max(n) <= 64
+            assert legal[s] == sum(n)
+            cnt = 0
+            for qt, x in enumerate(n):
+                wd = int(m[row + qt, 0])
+                assert int(m[row + qt, 1]) == wd                      # same word per KV head
+                assert wd >> x == 0                                   # no bits beyond legal groups
+                cnt += bin(wd).count("1")
+            K = (p * sum(n) + 50) // 100
+            assert cnt == K == int8[s]
+            assert abs(100.0 * cnt / sum(n) - p) <= 50.0 / sum(n) + 1e-9
+            if p == 0:
+                assert not m[row:row + len(n)].any()
+            if p == 100:
+                assert all(int(m[row + qt, 0]) == (1 << x) - 1 for qt, x in enumerate(n))
+            row += len(n)
+
+
+def _fp16_sets(template, p, n, seed=0):
+    return oracle.fp16_groups(template, p, seed, n)
+
+
+def test_template_structure():
+    n = [2 * qt + 2 for qt in range(32)]               # L = 4096, g = 1
+    for p in (25, 50, 75):
+        band = _fp16_sets("band", p, n)
+        glob = _fp16_sets("global", p, n)
+        al = _fp16_sets("aligned_sparse", p, n)
+        for x, b, gl, a in zip(n, band, glob, al):
+            assert b == set(range(x - len(b), x))             # suffix at the diagonal
+            assert gl == set(range(0, len(gl)))               # prefix at the sink keys
+            assert a == set(range(x - len(a), x))
+            if x >= 2:
+                assert {0, 1} <= gl
+        # Band is a fixed width: rows differ by at most one group (plus short rows)
+        widths = sorted({len(b) for x, b in zip(n, band) if x > len(b)})
+        assert len(widths) <= 2
+    # SpTrans at a full 64-group row and 75%: exactly residues {6, 7} of each 8
+    st = _fp16_sets("sptrans", 75, [64])
+    assert st[0] == {b for b in range(64) if b % 8 in (6, 7)}
+    # BigBird contains its leftmost and rightmost parts, and the random part varies
+    n = [64] * 4
+    bb0 = _fp16_sets("bigbird", 50, n, seed=1)
+    bb1 = _fp16_sets("bigbird", 50, n, seed=2)
+    for s in bb0:
+        f = len(s)
+        a = -(-f // 3)
+        b = -(-(f - a) // 2)
+        assert set(range(a)) <= s and set(range(64 - b, 64)) <= s
+    assert bb0 != bb1
+    rr = _fp16_sets("row_random", 25, n, seed=1)
+    assert all(len(s) == 48 for s in rr) and rr[0] != rr[1]
+
+
+def test_global_workload_width():
+    # 8k, g = 2, 75%: width 8 plus one extra for rows 8..43
+    n = [qt + 1 for qt in range(64)]
+    gl = _fp16_sets("global", 75, n)
+    for qt, s in enumerate(gl):
+        want = min(8, n[qt]) + (1 if 8 <= qt <= 43 else 0)
+        assert s == set(range(want))
+
+
+# --------------------------------------------------------------------------
+# attention pins
+# --------------------------------------------------------------------------
+
+SHAPES = [([64], 1, 1, 64), ([100], 1, 1, 64), ([256], 4, 2, 64), ([100, 200, 64], 4, 2, 64),
+          ([130], 2, 2, 128)]
+
+
+@pytest.mark.parametrize("lengths,hq,hk,d", SHAPES)
+@pytest.mark.parametrize("causal", [True, False])
+def test_all_fp16_equals_softmax_attention(lengths, hq, hk, d, causal):
+    inp = _inputs(lengths, hq, hk, d)
+    g = [1] * len(lengths)
+    O, lse = _run(inp, _words(lengths, hk, 0), g, lengths, causal)
+    Or, lr = bf.naive_attention(inp[0], inp[1], inp[2], lengths, causal)
+    assert np.abs(O - Or).max() < 1e-12
+    assert np.abs(lse - lr).max() < 1e-12
+
+
+@pytest.mark.parametrize("lengths,hq,hk,d", SHAPES)
+def test_all_int8_equals_uniform_int8(lengths, hq, hk, d):
+    inp = _inputs(lengths, hq, hk, d)
+    g = [1] * len(lengths)
+    ones = _words(lengths, hk, (1 << 64) - 1)
+    O, lse = _run(inp, ones, g, lengths, True)
+    Or, lr = bf.routed_attention(*inp, ones, g, lengths, True)
+    assert np.abs(O - Or).max() < 1e-12
+    assert np.abs(lse - lr).max() < 1e-12
+    # and it is really the INT8 path: it differs from the FP16 result
+    O0, _ = _run(inp, _words(lengths, hk, 0), g, lengths, True)
+    assert np.abs(O - O0).max() > 1e-6
+
+
+@pytest.mark.parametrize("g", [1, 2, 3])
+def test_mixed_words_equal_per_key_bruteforce(g):
+    lengths = [100, 300, 64]
+    hq, hk, d = 4, 2, 64
+    inp = _inputs(lengths, hq, hk, d, seed=9)
+    tm = sum(oracle.n_qtiles(L) for L in lengths)
+    rng = np.random.default_rng(g)
+    masks = rng.integers(0, 2 ** 63, size=(tm, hk), dtype=np.uint64) * np.uint64(2) + \
+        rng.integers(0, 2, size=(tm, hk), dtype=np.uint64)
+    gs = [g] * len(lengths)
+    for causal in (True, False):
+        O, lse = _run(inp, masks, gs, lengths, causal)
+        Or, lr = bf.routed_attention(*inp, masks, gs, lengths, causal)
+        assert np.abs(O - Or).max() < 1e-12
+        assert np.abs(lse - lr).max() < 1e-12
+
+
+def test_bits_beyond_legal_groups_are_ignored():
+    lengths = [300]
+    inp = _inputs(lengths, 2, 1, 64)
+    m, _, _ = oracle.build_routing("sptrans", 75, 0, lengths, 1, [1], True)
+    full = m.copy()
+    for qt in range(m.shape[0]):
+        n = oracle.legal_groups(qt, 300, 1, True)
+        full[qt] = np.uint64(int(m[qt, 0]) | (((1 << 64) - 1) ^ ((1 << n) - 1)))
+    a, _ = _run(inp, m, [1], lengths, True)
+    b, _ = _run(inp, full, [1], lengths, True)
+    assert np.array_equal(a, b)
+
+
+def test_illegal_entries_never_contribute():
+    # NaN in every K/V block after the last legal tile of q-tile row 0, and in
+    # the neighbouring sequences: rows 0..127 of the middle sequence unchanged.
+    lengths = [64, 384, 128]
+    hq, hk, d = 2, 1, 64
+    inp = list(_inputs(lengths, hq, hk, d))
+    m = oracle.build_routing("bigbird", 50, 1, lengths, hk, [1, 1, 1], True)[0]
+    base, _ = _run(inp, m, [1, 1, 1], lengths, True)
+    q, k, v = inp[0].copy(), inp[1].copy(), inp[2].copy()
+    t0 = 64
+    last = oracle.last_legal_tile(0, 384, True)         # = 1
+    k[t0 + (last + 1) * 64:t0 + 384] = np.nan
+    v[t0 + (last + 1) * 64:t0 + 384] = np.inf
+    k[:64] = np.nan
+    v[:64] = np.nan
+    k[448:] = np.nan
+    v[448:] = np.nan
+    q8, qs = oracle.quantize_q(q, lengths)
+    k8, ks = oracle.quantize_k(k, lengths)
+    got, _ = _run([q, k, v, q8, qs, k8, ks], m, [1, 1, 1], lengths, True)
+    assert np.isfinite(got[t0:t0 + 128]).all()
+    assert np.array_equal(got[t0:t0 + 128], base[t0:t0 + 128])
+
+
+def test_gqa_heads_share_their_kv_word():
+    lengths = [256, 130]
+    hq, hk, d = 4, 2, 64
+    inp = _inputs(lengths, hq, hk, d, seed=4)
+    tm = sum(oracle.n_qtiles(L) for L in lengths)
+    rng = np.random.default_rng(0)
+    masks = rng.integers(0, 16, size=(tm, hk), dtype=np.uint64)
+    assert (masks[:, 0] != masks[:, 1]).any()
+    g = [1, 1]
+    O, _ = _run(inp, masks, g, lengths, True)
+    q, k, v, q8, qs, k8, ks = inp
+    for h in range(hq):
+        kv = h // 2
+        sub = (q[:, h:h + 1], k[:, kv:kv + 1], v[:, kv:kv + 1], q8[:, h:h + 1], qs[h:h + 1],
+               k8[:, kv:kv + 1], ks[kv:kv + 1])
+        Oh, _ = _run(sub, masks[:, kv:kv + 1], g, lengths, True)
+        assert np.array_equal(Oh[:, 0], O[:, h])
+    # permuting query heads inside a KV group permutes the outputs
+    perm = [1, 0, 3, 2]
+    sub = (q[:, perm], k, v, q8[:, perm], qs[perm], k8, ks)
+    Op, _ = _run(sub, masks, g, lengths, True)
+    assert np.array_equal(Op, O[:, perm])
+
+
+def test_scale_exact_inputs_make_paths_agree():
+    # values c * 2^-5 with |c| <= 127 and one |c| = 127 in every block: the
+    # quantiser is exact, so INT8 and FP16 scores are the same real number.
+    lengths = [256, 100]
+    hq, hk, d = 2, 1, 64
+    T = sum(lengths)
+    rng = np.random.default_rng(11)
+
+    def codes(H):
+        c = rng.integers(-127, 128, size=(T, H, d))
+        for t in range(0, T, 64):
+            c[t, :, 0] = 127 * (1 if (t // 64) % 2 else -1)
+        return c
+
+    cq, ck = codes(hq), codes(hk)
+    q = (cq * 2.0 ** -5).astype(np.float16)
+    k = (ck * 2.0 ** -5).astype(np.float16)
+    v = rng.standard_normal((T, hk, d)).astype(np.float16)
+    q8, qs = oracle.quantize_q(q, lengths)
+    k8, ks = oracle.quantize_k(k, lengths)
+    assert np.array_equal(q8, cq) and np.array_equal(k8, ck)
+    assert (qs == np.float32(2.0 ** -5)).all() and (ks == np.float32(2.0 ** -5)).all()
+    inp = (q, k, v, q8, qs, k8, ks)
+    a, la = _run(inp, _words(lengths, hk, (1 << 64) - 1), [1, 1], lengths, True)
+    b, lb = _run(inp, _words(lengths, hk, 0), [1, 1], lengths, True)
+    assert np.abs(a - b).max() <= 1e-12 and np.abs(la - lb).max() <= 1e-12
+
+
+def test_int_scores_exact():
+    lengths = [200]
+    inp = _inputs(lengths, 1, 1, 64)
+    q8, k8 = inp[3], inp[5]
+    m = oracle.build_routing("band", 50, 0, lengths, 1, [1], True)[0]
+    A = oracle.int_scores(q8, k8, m, [1], lengths, 0, 0, 1, 1, True)
+    full = q8[:, 0].astype(np.int64) @ k8[:, 0].astype(np.int64).T
+    for i in range(200):
+        keys = bf.int8_keys_of_word(m[i // 128, 0], 200, 1)
+        for j in range(200):
+            if j <= i and keys[j]:
+                assert A[i, j] == full[i, j]
+            else:
+                assert A[i, j] == -(2 ** 62)
+    assert np.abs(full).max() < 2 ** 22
+
+
+def test_deviation_grows_with_coverage():
+    # not a parity pin: the trend the pages report (deviation from all-FP16
+    # rises with INT8 coverage), checked on one seeded case
+    lengths = [512]
+    inp = _inputs(lengths, 2, 1, 64, seed=2)
+    base, _ = _run(inp, _words(lengths, 1, 0), [1], lengths, True)
+    mads = []
+    for p in (0, 25, 50, 75, 100):
+        m = oracle.build_routing("sptrans", p, 0, lengths, 1, [1], True)[0]
+        O, _ = _run(inp, m, [1], lengths, True)
+        mads.append(np.abs(O - base).mean())
+    assert mads[0] == 0.0
+    assert all(b >= a for a, b in zip(mads, mads[1:]))
