@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Throughput of tile-routed FP16/INT8 causal prefill attention on B200.
+
+One step = one pass of the whole hot path over one batch: K block
+quantisation, Q block quantisation and the fused routed attention kernel,
+launched through the C ABI (tilemix_prefill_fwd).  Default workload: LLaMA-3.2-3B
+attention shape, batch 8 x 4096 tokens, 24 query / 8 KV heads, head dim 128,
+causal, SpTrans routing at 75% INT8 of legal tile groups, synthetic N(0,1)
+inputs with four x8 outlier channels per KV head.
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
+batch (weak scaling, no collective on the data path); timing is the max over
+ranks.  ``--impl reference`` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "attention prefill tok/s at 4k b8 (3B GQA shape); % of mixed tensor roofline"
+UNIT = "tok/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_F16 = 4.5 / 2.25  # nominal dense INT8 : FP16 tensor rate on B200
+
+
+# ----------------------------------------------------------------- helpers ---
+
+def workload(name, template=None, percent=None):
+    w = dict(synth.WORKLOADS[name])
+    if template:
+        w["template"] = template
+    if percent is not None:
+        w["percent"] = int(percent)
+    lengths = synth.workload_lengths(name)
+    if w["g"] == "auto":
+        g = [max(1, math.ceil(math.ceil(L / 64) / 64)) for L in lengths]
+    else:
+        g = [int(w["g"])] * len(lengths)
+    return w, lengths, g
+
+
+def legal_pairs(L, causal):
+    """[Tm, Tn] legal (query, key) pair counts of one sequence's tile grid."""
+    tm, tn = math.ceil(L / 128), math.ceil(L / 64)
+    out = np.zeros((tm, tn), dtype=np.int64)
+    for qt in range(tm):
+        rows = np.arange(qt * 128, min(L, qt * 128 + 128))
+        for kt in range(tn):
+            k0, k1 = kt * 64, min(L, kt * 64 + 64)
+            if causal:
+                out[qt, kt] = np.clip(rows - k0 + 1, 0, k1 - k0).sum()
+            else:
+                out[qt, kt] = len(rows) * (k1 - k0)
+    return out
+
+
+def algorithmic_work(lengths, hq, hk, d, masks, g, causal):
+    """FP16 FLOPs, INT8 ops and HBM bytes of one batch (legal pairs only:
+    2d per pair for QK in the routed precision, 2d FP16 for PV; bytes = Q, K,
+    V read once and O written once in fp16)."""
+    f16 = 0
+    i8 = 0
+    row = 0
+    group = hq // hk
+    for s, L in enumerate(lengths):
+        pairs = legal_pairs(L, causal)
+        for qt in range(pairs.shape[0]):
+            for kv in range(hk):
+                w = int(masks[row + qt, kv])
+                bits = np.array([(w >> (kt // g[s])) & 1 for kt in range(pairs.shape[1])], bool)
+                p_int = int(pairs[qt, bits].sum())
+                p_all = int(pairs[qt].sum())
+                i8 += group * 2 * d * p_int
+                f16 += group * 2 * d * (p_all - p_int) + group * 2 * d * p_all
+        row += pairs.shape[0]
+    T = sum(lengths)
+    nbytes = T * (2 * hq + 2 * hk) * d * 2
+    return f16, i8, nbytes
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of this GPU, every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", "tilemix_clocks_%d_%d.csv" % (os.getpid(), time.time_ns()))
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id,
+                                          "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------ oracle side ---
+
+def oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, rows, quant=None):
+    """Run the CPU oracle on `rows` and return (seconds, quant seconds)."""
+    import oracle
+    tq = 0.0
+    if quant is None:
+        t = time.perf_counter()
+        q8, qs = oracle.quantize_q(q, lengths)
+        k8, ks = oracle.quantize_k(k, lengths)
+        tq = time.perf_counter() - t
+        quant = (q8, qs, k8, ks)
+    q8, qs, k8, ks = quant
+    t = time.perf_counter()
+    oracle.attention_rows(q, k, v, q8, qs, k8, ks, masks, g, lengths, causal, rows=rows)
+    return time.perf_counter() - t, tq, quant
+
+
+def random_rows(lengths, hq, n, rng):
+    s = rng.integers(0, len(lengths), size=n)
+    h = rng.integers(0, hq, size=n)
+    L = np.asarray(lengths)[s]
+    i = (rng.random(n) * L).astype(np.int64)
+    return np.stack([s, h, i], axis=1).astype(np.int64)
+
+
+def cpu_baseline(q, k, v, lengths, hq, hk, masks, g, causal, budget_s=15.0):
+    """Oracle throughput on a bounded random-row sample, in prefill tokens/s
+    (one token = all hq heads of a row; quantisation cost charged pro rata)."""
+    rng = np.random.default_rng(1234)
+    T = sum(lengths)
+    cal = random_rows(lengths, hq, 256, rng)
+    t_cal, t_quant, quant = oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, cal)
+    n = int(max(256, min(200000, 256 * budget_s / max(t_cal, 1e-3))))
+    rows = random_rows(lengths, hq, n, rng)
+    t_rows, _, _ = oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, rows, quant=quant)
+    t = t_rows + t_quant * n / (T * hq)
+    return {"value": (n / hq) / t, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+            "sample": "%d uniformly random (sequence, head, row) outputs of the workload, fp64 "
+                      "oracle rows plus the numpy quantisation pro rata (%.1f s)" % (n, t)}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, timed step by step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w, lengths, g = workload(args.workload, args.template, args.percent)
+    hq, hk, d, causal = w["hq"], w["hk"], w["d"], w["causal"]
+    T = sum(lengths)
+    q, k, v = synth.make_qkv(0, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
+    import oracle
+    masks = oracle.build_routing(w["template"], w["percent"], w["routing_seed"], lengths, hk, g,
+                                 causal)[0]
+    rng = np.random.default_rng(99)
+    cal = random_rows(lengths, hq, 64, rng)
+    t_cal, t_quant, quant = oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, cal)
+    per_step_budget = max(0.02, 90.0 / max(1, args.steps + args.warmup))
+    n = int(max(16, min(100000, 64 * per_step_budget / max(t_cal, 1e-4))))
+    for _ in range(args.warmup):
+        oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, random_rows(lengths, hq, n, rng),
+                      quant=quant)
+    total = 0.0
+    for _ in range(args.steps):
+        rows = random_rows(lengths, hq, n, rng)
+        t, _, _ = oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, rows, quant=quant)
+        total += t + t_quant * n / (T * hq)
+    ms = 1e3 * total / args.steps
+    value = (n / hq) / (total / args.steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+i64",
+        "data": "synthetic", "config": bench_config(args, w, lengths, g),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                         "sample": "%d random (sequence, head, row) outputs per step" % n},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def bench_config(args, w, lengths, g):
+    return {"workload": args.workload, "batch": len(lengths), "seq_len": lengths[0]
+            if len(set(lengths)) == 1 else "varlen", "hq": w["hq"], "hk": w["hk"],
+            "head_dim": w["d"], "causal": w["causal"], "template": w["template"],
+            "int8_percent": w["percent"], "g": g[0] if len(set(g)) == 1 else "per-sequence",
+            "block_m": 128, "block_n": 64,
+            "l2": "no flush: inputs and output (%.0f MB per step) exceed the 126 MB L2"
+                  % (sum(lengths) * (2 * w["hq"] + 2 * w["hk"]) * w["d"] * 2 / 1e6)}
+
+
+# ---------------------------------------------------------------- GPU side ---
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import tile_routed_mixed_b200 as tm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w, lengths, g = workload(args.workload, args.template, args.percent)
+    hq, hk, d, causal = w["hq"], w["hk"], w["d"], w["causal"]
+    T = sum(lengths)
+    q, k, v = synth.make_qkv(rank, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
+    cu = synth.cu_seqlens_of(lengths)
+    masks, legal, int8 = tm.tilemix_build_routing(w["template"], w["percent"],
+                                                  w["routing_seed"], cu, hk, g, causal)
+    pf = tm.TileMixPrefill(lengths, hq, hk, d, masks, g, causal=causal, device=dev)
+    qd, kd, vd = (torch.from_numpy(x).to(dev) for x in (q, k, v))
+    od = torch.empty_like(qd)
+    pf.ensure_workspace(qd, kd, vd, od)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:  # torch creates the CUDA event on first record: force it now
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    args_plain = pf.args(qd, kd, vd, od)
+    args_timed = [pf.args(qd, kd, vd, od, events=e) for e in ev]
+
+    for _ in range(args.warmup):
+        tm.tilemix_prefill_fwd(args_plain, stream)
+    rc = tm.tilemix_get_error(stream)
+    if rc != tm.OK:
+        raise tm.TileMixError(rc, "warm-up")
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)  # let the sampler take its first sample
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        tm.tilemix_prefill_fwd(args_timed[i], stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    rc = tm.tilemix_get_error(stream)
+    if rc != tm.OK:
+        raise tm.TileMixError(rc, "timed steps")
+    ms = e0.elapsed_time(e1) / args.steps
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    t = torch.tensor([ms, kern_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, kern_ms = float(t[0]), float(t[1])
+
+    # end to end through the public call with pinned host buffers
+    qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        tm.tilemix_prefill_fwd(args_plain, stream)
+        oh.copy_(od, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        dist.destroy_process_group()
+    e2e_ms = float(t[0])
+    if rank != 0:
+        return
+
+    f16, i8, nbytes = algorithmic_work(lengths, hq, hk, d, masks, g, causal)
+    pk = peaks()
+    p16 = pk["bf16_tflops"] * 1e12
+    p8 = p16 * INT8_OVER_F16
+    t_tensor = f16 / p16 + i8 / p8
+    t_mem = nbytes / (pk["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_tensor >= t_mem else "hbm"
+    t_k = kern_ms / 1e3
+    if bound == "tensor":
+        achieved = (f16 + i8 * p16 / p8) / t_k / 1e12   # FP16-equivalent TFLOP/s
+        peak, unit = p16 / 1e12, "TFLOP/s"
+    else:
+        achieved, peak, unit = nbytes / t_k / 1e9, pk["hbm_gbs"], "GB/s"
+    tokens = T * world
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16+i8",
+        "data": "synthetic",
+        "config": bench_config(args, w, lengths, g),
+        "roofline": {
+            "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": None,
+            "kernel": "prefill_fwd_kernel<128>",
+            "kernel_ms": kern_ms,
+            "peak_kind": "burst (%s)" % pk["source"],
+            "fp16_flops": f16, "int8_ops": i8, "hbm_bytes": nbytes,
+            "mixed_roof_ms": 1e3 * max(t_tensor, t_mem),
+            "tflops_raw": (f16 + i8) / t_k / 1e12,
+            "int8_share_of_legal_groups": float(int8.sum() / legal.sum()),
+        },
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(q.nbytes + k.nbytes + v.nbytes),
+                "d2h_bytes_per_step": int(q.nbytes)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(q, k, v, lengths, hq, hk, masks, g, causal)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["tilemix", "reference"], default="tilemix")
+    ap.add_argument("--workload", default="llama3b_4k_b8", choices=list(synth.WORKLOADS))
+    ap.add_argument("--template", default=None)
+    ap.add_argument("--percent", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/* tilemix.h -- C ABI of the B200 (sm_100a) tile-routed FP16/INT8 causal
+ * prefill attention library (libtilemix.so).
+ *
+ * The method ("TileMix: Tile-Centric Mixed-Precision Attention for LLM
+ * Inference Acceleration", agihunt.info summary, method paragraphs; also
+ * "Precision Has a Map: TileMix Routes INT8 Inside Dense Attention",
+ * cognaptus.com, sections "Dense attention does not require uniform precision"
+ * and "The routing mechanism is designed to stay inside the hot loop"):
+ *   - the score matrix S = Q K^T of each (sequence, query head) is cut into
+ *     128 x 64 tiles (BLOCK_M query rows x BLOCK_N keys);
+ *   - g adjacent key tiles form one routing group; one bit per group, read by
+ *     shift-and-mask from one 64-bit word per (KV head, query-tile row);
+ *     bit 1 = INT8 score path, bit 0 = FP16 score path;
+ *   - INT8 path: Q quantised in 128 x d blocks and K in 64 x d blocks,
+ *     symmetric absmax / 127; INT8 MMA with INT32 accumulation; scores
+ *     rescaled by s_q * s_k / sqrt(d) into the float score domain;
+ *   - FP16 path: FP16 MMA with fp32 accumulation, scaled by 1 / sqrt(d);
+ *   - both paths update one online-softmax state (row max, normaliser,
+ *     output accumulator); V and P.V stay FP16;
+ *   - causal and boundary legality are applied independently of the routing
+ *     words: illegal interactions are never computed;
+ *   - GQA query heads read their KV head's word; batches are packed with
+ *     cu_seqlens (variable length, no padding).
+ *
+ * Conventions for every entry point:
+ *   - the return value is a tilemix_status; nothing throws or aborts;
+ *   - the caller owns every buffer; the library allocates no memory (host or
+ *     device) on any path;
+ *   - device entry points are asynchronous on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Argument errors are returned synchronously;
+ *     faults found on the device (a bounded wait that expired, a routing row
+ *     with more than 64 groups) are latched in a device status word and
+ *     returned by tilemix_get_error();
+ *   - "device" pointers must be CUDA device (or managed) memory of the current
+ *     device; "host" pointers are ordinary host memory.
+ */
+#ifndef TILEMIX_H
+#define TILEMIX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TILEMIX_VERSION 1
+#define TILEMIX_BLOCK_M 128  /* query rows per tile and per Q quantisation block */
+#define TILEMIX_BLOCK_N 64   /* keys per tile and per K quantisation block */
+#define TILEMIX_MAX_GROUPS 64
+
+typedef enum {
+  TILEMIX_OK = 0,
+  TILEMIX_ERR_INVALID_ARG = 1,  /* a pointer, size, layout or alignment is wrong */
+  TILEMIX_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. head dim not 64/128) */
+  TILEMIX_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  TILEMIX_ERR_TIMEOUT = 4,      /* a bounded device wait expired; outputs undefined */
+  TILEMIX_ERR_WORKSPACE = 5     /* workspace missing or smaller than required */
+} tilemix_status;
+
+typedef enum {
+  TILEMIX_BAND = 0,            /* keeps the diagonal local */
+  TILEMIX_GLOBAL = 1,          /* keeps designated (leftmost) positions */
+  TILEMIX_ROW_RANDOM = 2,      /* each row keeps random FP16 groups */
+  TILEMIX_ALIGNED_SPARSE = 3,  /* right-aligned FP16 extension */
+  TILEMIX_BIGBIRD = 4,         /* union of Band, Global and Row-Random */
+  TILEMIX_SPTRANS = 5          /* stride plus tail */
+} tilemix_template;
+
+/* Library version (TILEMIX_VERSION). */
+int tilemix_version(void);
+
+/* Static text for a tilemix_status value; never NULL. */
+const char* tilemix_status_string(int status);
+
+/* ---------------------------------------------------------------- host --- */
+
+/* Smallest grouping factor g >= 1 with ceil(ceil(seqlen / 64) / g) <= 64, so
+ * that every query-tile row of a sequence of `seqlen` tokens fits one 64-bit
+ * word (the grouping factor of the TileMix pages).  seqlen >= 0; g_out host.
+ * INVALID_ARG if g_out is NULL or seqlen < 0. */
+int tilemix_auto_g(int seqlen, int* g_out);
+
+/* Per-sequence tile offsets of a packed batch.  cu_seqlens_h (host, nseq+1,
+ * non-decreasing, starting at 0) -> cu_qtiles_h[s] = sum over s' < s of
+ * ceil(L_s' / 128) and cu_ktiles_h[s] = sum of ceil(L_s' / 64) (host, nseq+1
+ * each, caller-allocated).  INVALID_ARG on NULL pointers, nseq < 0 or
+ * decreasing offsets. */
+int tilemix_tile_offsets(const int32_t* cu_seqlens_h, int nseq, int32_t* cu_qtiles_h,
+                         int32_t* cu_ktiles_h);
+
+/* Routing words of a static template at a stated INT8 coverage of legal tile
+ * groups (TileMix pages: data-free templates borrowed from sparse attention;
+ * coverage is the share of legal groups routed INT8, not a FLOP share; the
+ * same words are reused for every KV head).
+ *   tpl            tilemix_template
+ *   int8_percent   0..100; per sequence exactly floor((p * N + 50) / 100) of
+ *                  its N legal groups are INT8
+ *   seed           seed of the Row-Random / BigBird draws (splitmix64)
+ *   cu_seqlens_h   host [nseq+1]
+ *   n_kv_heads     >= 1
+ *   g_h            host [nseq], grouping factor per sequence (>= 1); a row with
+ *                  more than 64 legal groups is INVALID_ARG
+ *   causal         0 or 1
+ *   masks_h        host [total_qtiles][n_kv_heads] uint64, caller-allocated;
+ *                  bit b (LSB first) = group b (key tiles [b*g, (b+1)*g)),
+ *                  1 = INT8; bits at and above a row's legal group count are 0
+ *   legal_groups_h host [nseq] or NULL: N per sequence
+ *   int8_groups_h  host [nseq] or NULL: INT8 groups per sequence
+ * The template geometries are stated in the repository's design notes. */
+int tilemix_build_routing(int tpl, int int8_percent, uint64_t seed, const int32_t* cu_seqlens_h,
+                          int nseq, int n_kv_heads, const int32_t* g_h, int causal,
+                          uint64_t* masks_h, int64_t* legal_groups_h, int64_t* int8_groups_h);
+
+/* -------------------------------------------------------------- device --- */
+
+/* Block quantisation of the INT8 score path (TileMix pages: only Q and K are
+ * quantised, Q per 128 x d block, K per 64 x d block, symmetric absmax / 127).
+ * Per (head, block of one sequence): a = max |x| over the block's valid rows,
+ * s = fp32(a / 127) (IEEE division), code = clamp(rne(fp32(x / s)), -127, 127);
+ * a == 0 gives s = 0 and codes 0.  Blocks start at each sequence's first token.
+ *   q_f16 / k_f16   device fp16 [total_tokens][hq or hk][d], 16-byte aligned;
+ *                   either may be NULL to skip that tensor (its outputs too)
+ *   cu_seqlens_d, cu_qtiles_d, cu_ktiles_d   device int32 [nseq+1]
+ *   q_i8            device int8 [total_tokens][hq][d]
+ *   q_scale         device fp32 [hq][total_qtiles]
+ *   k_i8            device int8 [total_tokens][hk][d]
+ *   k_scale         device fp32 [hk][total_ktiles]
+ *   d               64 or 128 (UNSUPPORTED otherwise) */
+int tilemix_quantize_qk(const void* q_f16, const void* k_f16, const int32_t* cu_seqlens_d,
+                        const int32_t* cu_qtiles_d, const int32_t* cu_ktiles_d, int nseq,
+                        int total_tokens, int total_qtiles, int total_ktiles, int hq, int hk,
+                        int d, int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                        void* stream);
+
+typedef struct tilemix_prefill_args {
+  const void* q;          /* device fp16 [total_tokens][hq][d], 16-byte aligned */
+  const void* k;          /* device fp16 [total_tokens][hk][d], 16-byte aligned */
+  const void* v;          /* device fp16 [total_tokens][hk][d], 16-byte aligned */
+  void* o;                /* device fp16 [total_tokens][hq][d], 16-byte aligned (output) */
+  float* lse;             /* device fp32 [hq][total_tokens] natural-log LSE, or NULL */
+  const int32_t* cu_seqlens; /* device [nseq+1], packed token offsets */
+  const int32_t* cu_qtiles;  /* device [nseq+1], see tilemix_tile_offsets */
+  const int32_t* cu_ktiles;  /* device [nseq+1] */
+  int nseq;
+  int total_tokens;       /* cu_seqlens[nseq] */
+  int total_qtiles;       /* cu_qtiles[nseq] */
+  int total_ktiles;       /* cu_ktiles[nseq] */
+  int max_seqlen;         /* max L_s (upper bound accepted) */
+  int hq, hk, d;          /* hq % hk == 0; d in {64, 128} */
+  const int32_t* kv_head_of_q; /* device [hq], or NULL for h / (hq / hk) */
+  const uint64_t* masks;  /* device [total_qtiles][hk] routing words */
+  const int32_t* g;       /* device [nseq] grouping factors */
+  int causal;             /* 1: key j legal for query i iff j <= i (and j < L_s) */
+  float softmax_scale;    /* 0 selects 1 / sqrt(d) */
+  const int8_t* k_i8;     /* optional precomputed K codes [total_tokens][hk][d] ... */
+  const float* k_scale;   /* ... and scales [hk][total_ktiles]; both or neither */
+  void* workspace;        /* device scratch, >= tilemix_workspace_size(), 256-aligned */
+  size_t workspace_bytes;
+  int32_t* debug_int32_scores; /* NULL, or device int32 [hq][total_tokens][dbg_cols]
+                                  with dbg_cols = max_seqlen rounded up to 64: the raw
+                                  INT32 score of every INT8-routed key tile computed
+                                  (keys < L_s; other entries untouched).  Small
+                                  inputs only; slows the kernel. */
+  void* event_kernel_begin;    /* NULL, or a cudaEvent_t recorded on `stream` just
+                                  before the fused attention kernel ... */
+  void* event_kernel_end;      /* ... and one recorded just after it (profiling) */
+} tilemix_prefill_args;
+
+/* Bytes of device workspace tilemix_prefill_fwd needs for these arguments
+ * (it holds the INT8 codes and scales of Q, and of K unless k_i8 is given).
+ * INVALID_ARG on a NULL argument. */
+int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes);
+
+/* Fused tile-routed mixed-precision causal prefill attention forward:
+ * O[t, h] = softmax over legal keys of the routed scores, times V, in fp16
+ * (one rounding of the fp32 accumulator divided by the normaliser).
+ * Enqueues the K quantisation pre-pass (unless k_i8 is given), the Q
+ * quantisation and the fused attention kernel on `stream`. */
+int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * OK, TIMEOUT (a bounded wait expired), INVALID_ARG (a row needed more than 64
+ * groups, or a bad routing-group factor), or CUDA for a sticky CUDA error. */
+int tilemix_get_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILEMIX_H */

@@ -1,0 +1,142 @@
+"""The C-ABI library: load, exported symbols, host-side helpers against the
+oracle, and synchronous argument checks.  No GPU needed (no device calls)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+import tile_routed_mixed_b200 as tm
+from tile_routed_mixed_b200 import build as tmbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    tmbuild.build()
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "tilemix.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tilemix_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert "tilemix_prefill_fwd" in names and len(names) >= 9
+    L = ctypes.CDLL(tm.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    assert tm.tilemix_version() == 1
+    assert tm.status_string(tm.ERR_TIMEOUT) == "device wait timed out"
+
+
+def test_auto_g_and_offsets_match_oracle():
+    for L in (0, 1, 63, 64, 65, 4096, 4097, 8192, 12096, 16384, 65536, 65537):
+        assert tm.tilemix_auto_g(L) == oracle.auto_g(L)
+    lengths = [100, 0, 256, 64, 4097]
+    cu = synth.cu_seqlens_of(lengths)
+    cq, ck = tm.tilemix_tile_offsets(cu)
+    oq, ok = oracle.tile_offsets(lengths)
+    assert np.array_equal(cq, oq) and np.array_equal(ck, ok)
+
+
+def _geometries():
+    out = []
+    for name in synth.WORKLOADS:
+        w = synth.WORKLOADS[name]
+        lengths = synth.workload_lengths(name)
+        g = ([oracle.auto_g(L) for L in lengths] if w["g"] == "auto"
+             else [int(w["g"])] * len(lengths))
+        out.append((name, lengths, g, True))
+    out.append(("ragged", [100, 300, 1, 513, 2000], [1, 1, 1, 1, 1], True))
+    out.append(("ragged_noncausal", [100, 300, 513], [1, 1, 1], False))
+    out.append(("g3", [5000, 3000], [3, 2], True))
+    return out
+
+
+@pytest.mark.parametrize("geom", _geometries(), ids=lambda g: g[0])
+@pytest.mark.parametrize("template", list(tm.TEMPLATES))
+def test_routing_builder_bit_exact_vs_oracle(geom, template):
+    _, lengths, g, causal = geom
+    cu = synth.cu_seqlens_of(lengths)
+    for p in (0, 10, 25, 50, 75, 90, 100):
+        for seed in (0, 12345):
+            m, legal, int8 = tm.tilemix_build_routing(template, p, seed, cu, 3, g, causal)
+            mo, lo, io = oracle.build_routing(template, p, seed, lengths, 3, g, causal)
+            assert np.array_equal(m, mo), (template, p, seed)
+            assert np.array_equal(legal, lo) and np.array_equal(int8, io)
+
+
+def test_routing_builder_rejects_bad_arguments():
+    cu = synth.cu_seqlens_of([8192])
+    with pytest.raises(tm.TileMixError) as e:
+        tm.tilemix_build_routing("band", 50, 0, cu, 1, [1], True)   # 128 groups in a row
+    assert e.value.status == tm.ERR_INVALID_ARG
+    for bad in (-1, 101):
+        with pytest.raises(tm.TileMixError):
+            tm.tilemix_build_routing("band", bad, 0, cu, 1, [2], True)
+    with pytest.raises(tm.TileMixError):
+        tm.tilemix_build_routing(7, 50, 0, cu, 1, [2], True)
+    with pytest.raises(tm.TileMixError):
+        tm.tilemix_build_routing("band", 50, 0, cu, 0, [2], True)
+    with pytest.raises(tm.TileMixError):
+        tm.tilemix_build_routing("band", 50, 0, cu, 1, [0], True)
+    L = tm.lib()
+    assert L.tilemix_auto_g(-1, ctypes.byref(ctypes.c_int())) == tm.ERR_INVALID_ARG
+    assert L.tilemix_auto_g(5, None) == tm.ERR_INVALID_ARG
+    bad_cu = np.array([0, 10, 5], dtype=np.int32)
+    q = np.zeros(3, np.int32)
+    assert L.tilemix_tile_offsets(bad_cu.ctypes.data, 2, q.ctypes.data, q.ctypes.data) == \
+        tm.ERR_INVALID_ARG
+
+
+def _fake_args(**over):
+    a = tm.PrefillArgs()
+    a.q = a.k = a.v = a.o = 4096
+    a.cu_seqlens = a.cu_qtiles = a.cu_ktiles = a.masks = a.g = 4096
+    a.nseq, a.total_tokens, a.total_qtiles, a.total_ktiles, a.max_seqlen = 1, 256, 2, 4, 256
+    a.hq, a.hk, a.d = 4, 2, 128
+    a.causal = 1
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_prefill_argument_checks_are_synchronous():
+    L = tm.lib()
+    n = ctypes.c_size_t(0)
+    assert L.tilemix_workspace_size(ctypes.byref(_fake_args()), ctypes.byref(n)) == tm.OK
+    # q8 [256*4*128] + q scales [4*2 floats] + k8 [256*2*128] + k scales, each 256-aligned
+    assert n.value == 131072 + 256 + 65536 + 256
+    assert L.tilemix_workspace_size(ctypes.byref(_fake_args(k_i8=4096, k_scale=4096)),
+                                    ctypes.byref(n)) == tm.OK
+    assert n.value == 131072 + 256
+    cases = [
+        (dict(d=96), tm.ERR_UNSUPPORTED),
+        (dict(hq=3, hk=2), tm.ERR_INVALID_ARG),
+        (dict(hk=0), tm.ERR_INVALID_ARG),
+        (dict(causal=2), tm.ERR_INVALID_ARG),
+        (dict(q=None), tm.ERR_INVALID_ARG),
+        (dict(masks=None), tm.ERR_INVALID_ARG),
+        (dict(q=4100), tm.ERR_INVALID_ARG),            # not 16-byte aligned
+        (dict(k_i8=4096), tm.ERR_INVALID_ARG),         # codes without scales
+        (dict(softmax_scale=-1.0), tm.ERR_INVALID_ARG),
+        (dict(max_seqlen=0), tm.ERR_INVALID_ARG),
+        (dict(), tm.ERR_WORKSPACE),                    # no workspace given
+        (dict(workspace=4096, workspace_bytes=10), tm.ERR_WORKSPACE),
+        (dict(workspace=4100, workspace_bytes=1 << 30), tm.ERR_WORKSPACE),
+    ]
+    for over, want in cases:
+        assert L.tilemix_prefill_fwd(ctypes.byref(_fake_args(**over)), None) == want, over
+    # empty batches are a no-op
+    assert L.tilemix_prefill_fwd(ctypes.byref(_fake_args(nseq=0)), None) == tm.OK
+    assert L.tilemix_quantize_qk(None, None, None, None, None, 0, 0, 0, 0, 1, 1, 128, None, None,
+                                 None, None, None) == tm.OK
+    assert L.tilemix_quantize_qk(None, None, None, None, None, 1, 10, 1, 1, 1, 1, 80, None,
+                                 None, None, None, None) == tm.ERR_UNSUPPORTED

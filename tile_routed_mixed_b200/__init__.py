@@ -1,0 +1,226 @@
+"""Python binding of libtilemix.so: tile-routed FP16/INT8 causal prefill
+attention for B200 (sm_100a).
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+library.  PyTorch supplies device memory and streams.  If the library is
+missing this module raises on first use; there is no fallback.
+
+Names mirror the C ABI of ``include/tilemix.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtilemix.so")
+
+BLOCK_M = 128
+BLOCK_N = 64
+MAX_GROUPS = 64
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
+TEMPLATES = {"band": 0, "global": 1, "row_random": 2, "aligned_sparse": 3, "bigbird": 4,
+             "sptrans": 5}
+
+
+class TileMixError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+class PrefillArgs(ctypes.Structure):
+    """Mirror of ``tilemix_prefill_args``."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("cu_seqlens", ctypes.c_void_p), ("cu_qtiles", ctypes.c_void_p),
+        ("cu_ktiles", ctypes.c_void_p),
+        ("nseq", ctypes.c_int), ("total_tokens", ctypes.c_int), ("total_qtiles", ctypes.c_int),
+        ("total_ktiles", ctypes.c_int), ("max_seqlen", ctypes.c_int),
+        ("hq", ctypes.c_int), ("hk", ctypes.c_int), ("d", ctypes.c_int),
+        ("kv_head_of_q", ctypes.c_void_p), ("masks", ctypes.c_void_p), ("g", ctypes.c_void_p),
+        ("causal", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+        ("k_i8", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("debug_int32_scores", ctypes.c_void_p),
+        ("event_kernel_begin", ctypes.c_void_p), ("event_kernel_end", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libtilemix.so is missing at %s: run "
+                              "`python -m tile_routed_mixed_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        L.tilemix_version.restype = I
+        L.tilemix_status_string.restype = ctypes.c_char_p
+        L.tilemix_status_string.argtypes = [I]
+        L.tilemix_auto_g.restype = I
+        L.tilemix_auto_g.argtypes = [I, P]
+        L.tilemix_tile_offsets.restype = I
+        L.tilemix_tile_offsets.argtypes = [P, I, P, P]
+        L.tilemix_build_routing.restype = I
+        L.tilemix_build_routing.argtypes = [I, I, ctypes.c_uint64, P, I, I, P, I, P, P, P]
+        L.tilemix_quantize_qk.restype = I
+        L.tilemix_quantize_qk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P]
+        L.tilemix_workspace_size.restype = I
+        L.tilemix_workspace_size.argtypes = [ctypes.POINTER(PrefillArgs),
+                                             ctypes.POINTER(ctypes.c_size_t)]
+        L.tilemix_prefill_fwd.restype = I
+        L.tilemix_prefill_fwd.argtypes = [ctypes.POINTER(PrefillArgs), P]
+        L.tilemix_get_error.restype = I
+        L.tilemix_get_error.argtypes = [P]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().tilemix_status_string(int(status)).decode()
+
+
+tilemix_status_string = status_string
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise TileMixError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------------- host ---
+
+def tilemix_version() -> int:
+    return int(lib().tilemix_version())
+
+
+def tilemix_auto_g(seqlen: int) -> int:
+    g = ctypes.c_int(0)
+    _check(lib().tilemix_auto_g(int(seqlen), ctypes.byref(g)), "tilemix_auto_g")
+    return g.value
+
+
+def tilemix_tile_offsets(cu_seqlens):
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    nseq = cu.size - 1
+    cq = np.zeros(nseq + 1, dtype=np.int32)
+    ck = np.zeros(nseq + 1, dtype=np.int32)
+    _check(lib().tilemix_tile_offsets(cu.ctypes.data, nseq, cq.ctypes.data, ck.ctypes.data),
+           "tilemix_tile_offsets")
+    return cq, ck
+
+
+def tilemix_build_routing(template, int8_percent: int, seed: int, cu_seqlens, n_kv_heads: int,
+                          g, causal: bool = True):
+    """Routing words [total_qtiles, n_kv_heads] (uint64) and per-sequence
+    (legal groups, INT8 groups)."""
+    tpl = TEMPLATES[template] if isinstance(template, str) else int(template)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    nseq = cu.size - 1
+    gg = np.ascontiguousarray(g, dtype=np.int32)
+    if gg.size != nseq:
+        raise ValueError("one grouping factor per sequence")
+    cq, _ = tilemix_tile_offsets(cu)
+    masks = np.zeros((int(cq[-1]), int(n_kv_heads)), dtype=np.uint64)
+    legal = np.zeros(nseq, dtype=np.int64)
+    int8 = np.zeros(nseq, dtype=np.int64)
+    _check(lib().tilemix_build_routing(tpl, int(int8_percent), ctypes.c_uint64(seed & (2**64 - 1)),
+                                       cu.ctypes.data, nseq, int(n_kv_heads), gg.ctypes.data,
+                                       int(bool(causal)), masks.ctypes.data, legal.ctypes.data,
+                                       int8.ctypes.data),
+           "tilemix_build_routing")
+    return masks, legal, int8
+
+
+# ----------------------------------------------------------------- device ---
+
+def tilemix_quantize_qk(q, k, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_tokens,
+                        total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8, k_scale,
+                        stream=None):
+    _check(lib().tilemix_quantize_qk(_ptr(q), _ptr(k), _ptr(cu_seqlens), _ptr(cu_qtiles),
+                                     _ptr(cu_ktiles), int(nseq), int(total_tokens),
+                                     int(total_qtiles), int(total_ktiles), int(hq), int(hk),
+                                     int(d), _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
+                                     _ptr(k_scale), _stream_handle(stream)),
+           "tilemix_quantize_qk")
+
+
+def make_args(q, k, v, o, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_tokens, total_qtiles,
+              total_ktiles, max_seqlen, masks, g, causal=True, softmax_scale=0.0,
+              kv_head_of_q=None, lse=None, k_i8=None, k_scale=None, workspace=None,
+              debug_int32_scores=None, events=None) -> PrefillArgs:
+    T, hq, d = q.shape
+    hk = k.shape[1]
+    a = PrefillArgs()
+    a.q, a.k, a.v, a.o = (x.data_ptr() for x in (q, k, v, o))
+    a.lse = lse.data_ptr() if lse is not None else None
+    a.cu_seqlens, a.cu_qtiles, a.cu_ktiles = (x.data_ptr() for x in (cu_seqlens, cu_qtiles,
+                                                                       cu_ktiles))
+    a.nseq, a.total_tokens, a.total_qtiles, a.total_ktiles = (int(nseq), int(total_tokens),
+                                                               int(total_qtiles),
+                                                               int(total_ktiles))
+    a.max_seqlen = int(max_seqlen)
+    a.hq, a.hk, a.d = int(hq), int(hk), int(d)
+    a.kv_head_of_q = kv_head_of_q.data_ptr() if kv_head_of_q is not None else None
+    a.masks = masks.data_ptr()
+    a.g = g.data_ptr()
+    a.causal = int(bool(causal))
+    a.softmax_scale = float(softmax_scale)
+    a.k_i8 = k_i8.data_ptr() if k_i8 is not None else None
+    a.k_scale = k_scale.data_ptr() if k_scale is not None else None
+    if workspace is not None:
+        a.workspace = workspace.data_ptr()
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a.debug_int32_scores = (debug_int32_scores.data_ptr()
+                            if debug_int32_scores is not None else None)
+    if events is not None:  # (begin, end) torch.cuda.Event pair around the fused kernel
+        a.event_kernel_begin = events[0].cuda_event
+        a.event_kernel_end = events[1].cuda_event
+    return a
+
+
+def tilemix_workspace_size(args: PrefillArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tilemix_workspace_size(ctypes.byref(args), ctypes.byref(n)),
+           "tilemix_workspace_size")
+    return int(n.value)
+
+
+def tilemix_prefill_fwd(args: PrefillArgs, stream=None):
+    _check(lib().tilemix_prefill_fwd(ctypes.byref(args), _stream_handle(stream)),
+           "tilemix_prefill_fwd")
+
+
+def tilemix_get_error(stream=None) -> int:
+    return int(lib().tilemix_get_error(_stream_handle(stream)))
+
+
+from .prefill import TileMixPrefill  # noqa: E402  (convenience wrapper)
+
+__all__ = [
+    "BLOCK_M", "BLOCK_N", "MAX_GROUPS", "PrefillArgs", "TEMPLATES", "TileMixError",
+    "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
+    "tilemix_build_routing", "tilemix_get_error", "tilemix_prefill_fwd", "tilemix_quantize_qk",
+    "tilemix_status_string", "tilemix_tile_offsets", "tilemix_version",
+    "tilemix_workspace_size",
+]

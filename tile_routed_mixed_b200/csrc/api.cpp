@@ -1,0 +1,253 @@
+// Host side of the C ABI: argument checks, workspace layout, TMA descriptor
+// encoding and the kernel launch sequence.  Allocates no memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "tilemix.h"
+#include "tilemix_internal.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long ns = [] {
+    const char* env = std::getenv("TILEMIX_WAIT_TIMEOUT_MS");
+    long long ms = env ? std::atoll(env) : 2000;
+    if (ms < 1) ms = 1;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return ns;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Packed [rows][heads][d] tensor as a 3-D TMA map {d, heads, rows} with a box
+// of {box_inner, 1, box_rows} elements and the given swizzle.
+int encode_rows(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                int rows, int heads, int d, int box_inner, int box_rows,
+                CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return TILEMIX_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
+                                 static_cast<cuuint64_t>(d) * heads * elem_bytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1u,
+                             static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TILEMIX_OK : TILEMIX_ERR_CUDA;
+}
+
+struct WorkspaceLayout {
+  size_t q8, q_scale, k8, k_scale, total;
+};
+
+WorkspaceLayout layout_of(const tilemix_prefill_args* a) {
+  WorkspaceLayout w{};
+  const size_t T = static_cast<size_t>(a->total_tokens);
+  size_t off = 0;
+  w.q8 = off;
+  off = round_up(off + T * a->hq * a->d, 256);
+  w.q_scale = off;
+  off = round_up(off + sizeof(float) * a->hq * static_cast<size_t>(a->total_qtiles), 256);
+  const bool own_k = a->k_i8 == nullptr;
+  w.k8 = off;
+  if (own_k) off = round_up(off + T * a->hk * a->d, 256);
+  w.k_scale = off;
+  if (own_k) off = round_up(off + sizeof(float) * a->hk * static_cast<size_t>(a->total_ktiles), 256);
+  w.total = off;
+  return w;
+}
+
+int check_args(const tilemix_prefill_args* a) {
+  if (!a) return TILEMIX_ERR_INVALID_ARG;
+  if (a->d != 64 && a->d != 128) return TILEMIX_ERR_UNSUPPORTED;
+  if (a->hq < 1 || a->hk < 1 || a->hq % a->hk != 0) return TILEMIX_ERR_INVALID_ARG;
+  if (a->nseq < 0 || a->total_tokens < 0 || a->total_qtiles < 0 || a->total_ktiles < 0 ||
+      a->max_seqlen < 0)
+    return TILEMIX_ERR_INVALID_ARG;
+  if (a->causal != 0 && a->causal != 1) return TILEMIX_ERR_INVALID_ARG;
+  if (!(a->softmax_scale >= 0.f) || std::isinf(a->softmax_scale)) return TILEMIX_ERR_INVALID_ARG;
+  if ((a->k_i8 == nullptr) != (a->k_scale == nullptr)) return TILEMIX_ERR_INVALID_ARG;
+  if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;  // nothing to do
+  if (!a->q || !a->k || !a->v || !a->o || !a->cu_seqlens || !a->cu_qtiles || !a->cu_ktiles ||
+      !a->masks || !a->g)
+    return TILEMIX_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o) ||
+      (a->k_i8 && !aligned16(a->k_i8)))
+    return TILEMIX_ERR_INVALID_ARG;
+  if (a->max_seqlen < 1) return TILEMIX_ERR_INVALID_ARG;
+  return TILEMIX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+TILEMIX_API int tilemix_version(void) { return TILEMIX_VERSION; }
+
+TILEMIX_API const char* tilemix_status_string(int status) {
+  switch (status) {
+    case TILEMIX_OK: return "ok";
+    case TILEMIX_ERR_INVALID_ARG: return "invalid argument";
+    case TILEMIX_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TILEMIX_ERR_CUDA: return "CUDA error";
+    case TILEMIX_ERR_TIMEOUT: return "device wait timed out";
+    case TILEMIX_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+TILEMIX_API int tilemix_quantize_qk(const void* q_f16, const void* k_f16,
+                                    const int32_t* cu_seqlens_d, const int32_t* cu_qtiles_d,
+                                    const int32_t* cu_ktiles_d, int nseq, int total_tokens,
+                                    int total_qtiles, int total_ktiles, int hq, int hk, int d,
+                                    int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                                    void* stream) {
+  if (d != 64 && d != 128) return TILEMIX_ERR_UNSUPPORTED;
+  if (nseq < 0 || total_tokens < 0 || total_qtiles < 0 || total_ktiles < 0)
+    return TILEMIX_ERR_INVALID_ARG;
+  if (nseq == 0 || total_tokens == 0) return TILEMIX_OK;
+  if (!cu_seqlens_d) return TILEMIX_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (q_f16) {
+    if (hq < 1 || !cu_qtiles_d || !q_i8 || !q_scale || !aligned16(q_f16) ||
+        (reinterpret_cast<uintptr_t>(q_i8) & 7u))
+      return TILEMIX_ERR_INVALID_ARG;
+    if (tilemix::launch_quantize(q_f16, cu_seqlens_d, cu_qtiles_d, nseq, total_qtiles, hq, d,
+                                 TILEMIX_BLOCK_M, q_i8, q_scale, st) != cudaSuccess)
+      return TILEMIX_ERR_CUDA;
+  }
+  if (k_f16) {
+    if (hk < 1 || !cu_ktiles_d || !k_i8 || !k_scale || !aligned16(k_f16) ||
+        (reinterpret_cast<uintptr_t>(k_i8) & 7u))
+      return TILEMIX_ERR_INVALID_ARG;
+    if (tilemix::launch_quantize(k_f16, cu_seqlens_d, cu_ktiles_d, nseq, total_ktiles, hk, d,
+                                 TILEMIX_BLOCK_N, k_i8, k_scale, st) != cudaSuccess)
+      return TILEMIX_ERR_CUDA;
+  }
+  return TILEMIX_OK;
+}
+
+TILEMIX_API int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes) {
+  if (!args || !bytes) return TILEMIX_ERR_INVALID_ARG;
+  const int rc = check_args(args);
+  if (rc != TILEMIX_OK) return rc;
+  *bytes = layout_of(args).total;
+  return TILEMIX_OK;
+}
+
+TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream) {
+  int rc = check_args(a);
+  if (rc != TILEMIX_OK) return rc;
+  if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;
+  const WorkspaceLayout w = layout_of(a);
+  if (!a->workspace || a->workspace_bytes < w.total ||
+      (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return TILEMIX_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  int8_t* q8 = reinterpret_cast<int8_t*>(ws + w.q8);
+  float* q_scale = reinterpret_cast<float*>(ws + w.q_scale);
+  const int8_t* k8 = a->k_i8 ? a->k_i8 : reinterpret_cast<int8_t*>(ws + w.k8);
+  const float* k_scale = a->k_i8 ? a->k_scale : reinterpret_cast<float*>(ws + w.k_scale);
+
+  // INT8 path operands: Q always, K unless the caller supplied its codes.
+  rc = tilemix_quantize_qk(a->q, a->k_i8 ? nullptr : a->k, a->cu_seqlens, a->cu_qtiles,
+                           a->cu_ktiles, a->nseq, a->total_tokens, a->total_qtiles,
+                           a->total_ktiles, a->hq, a->hk, a->d, q8, q_scale,
+                           const_cast<int8_t*>(k8), const_cast<float*>(k_scale), stream);
+  if (rc != TILEMIX_OK) return rc;
+
+  tilemix::PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int T = a->total_tokens, d = a->d;
+  const CUtensorMapSwizzle sw8 =
+      d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if ((rc = encode_rows(&p.tm_q, a->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hq, d, 64,
+                        TILEMIX_BLOCK_M, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_q8, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a->hq, d, d,
+                        TILEMIX_BLOCK_M, sw8)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hk, d, 64,
+                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_k8, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a->hk, d, d,
+                        TILEMIX_BLOCK_N, sw8)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hk, d, 64,
+                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
+  p.o = a->o;
+  p.lse = a->lse;
+  p.cu_seqlens = a->cu_seqlens;
+  p.cu_qtiles = a->cu_qtiles;
+  p.cu_ktiles = a->cu_ktiles;
+  p.kv_head_of_q = a->kv_head_of_q;
+  p.masks = a->masks;
+  p.g = a->g;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.dbg = a->debug_int32_scores;
+  p.dbg_cols = (a->max_seqlen + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N * TILEMIX_BLOCK_N;
+  p.nseq = a->nseq;
+  p.total_tokens = T;
+  p.total_qtiles = a->total_qtiles;
+  p.total_ktiles = a->total_ktiles;
+  p.max_qtiles = (a->max_seqlen + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M;
+  p.hq = a->hq;
+  p.hk = a->hk;
+  p.group = a->hq / a->hk;
+  p.causal = a->causal;
+  const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = wait_timeout_ns();
+  if (a->event_kernel_begin &&
+      cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_begin), st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  if (tilemix::launch_prefill(p, d, st) != cudaSuccess) return TILEMIX_ERR_CUDA;
+  if (a->event_kernel_end &&
+      cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_end), st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  return TILEMIX_OK;
+}
+
+TILEMIX_API int tilemix_get_error(void* stream) {
+  unsigned int status = 0;
+  if (tilemix::read_and_clear_status(&status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  if (status & tilemix::kStatusTimeout) return TILEMIX_ERR_TIMEOUT;
+  if (status & tilemix::kStatusBadGroups) return TILEMIX_ERR_INVALID_ARG;
+  return TILEMIX_OK;
+}
+
+}  // extern "C"

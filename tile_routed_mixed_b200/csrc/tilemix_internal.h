@@ -1,0 +1,52 @@
+// Internal declarations shared by the host API and the kernel translation unit.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#define TILEMIX_API __attribute__((visibility("default")))
+
+namespace tilemix {
+
+// Bits of the device status word.
+enum : unsigned int {
+  kStatusTimeout = 1u,       // a bounded mbarrier wait expired
+  kStatusBadGroups = 2u,     // a row needed a routing group index above 63
+};
+
+// Everything the fused attention kernel needs, by value (kernel parameter).
+struct PrefillParams {
+  CUtensorMap tm_q;    // fp16 Q   [T][hq][d], box {64, 1, 128}, 128B swizzle
+  CUtensorMap tm_q8;   // int8 Q   [T][hq][d], box {d, 1, 128}
+  CUtensorMap tm_k;    // fp16 K   [T][hk][d], box {64, 1, 64}
+  CUtensorMap tm_k8;   // int8 K   [T][hk][d], box {d, 1, 64}
+  CUtensorMap tm_v;    // fp16 V   [T][hk][d], box {64, 1, 64}
+  void* o;
+  float* lse;
+  const int32_t* cu_seqlens;
+  const int32_t* cu_qtiles;
+  const int32_t* cu_ktiles;
+  const int32_t* kv_head_of_q;
+  const uint64_t* masks;
+  const int32_t* g;
+  const float* q_scale;   // [hq][total_qtiles]
+  const float* k_scale;   // [hk][total_ktiles]
+  int32_t* dbg;
+  int dbg_cols;
+  int nseq, total_tokens, total_qtiles, total_ktiles, max_qtiles;
+  int hq, hk, group;      // group = hq / hk
+  int causal;
+  float scale_log2;       // softmax scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+// Launchers implemented in the CUDA translation unit.  Return cudaError_t.
+int launch_quantize(const void* x, const int32_t* cu_seqlens, const int32_t* cu_tiles, int nseq,
+                    int total_tiles, int heads, int d, int block_rows, int8_t* codes,
+                    float* scales, cudaStream_t stream);
+int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
+int read_and_clear_status(unsigned int* status, cudaStream_t stream);
+
+}  // namespace tilemix

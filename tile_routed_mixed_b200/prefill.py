@@ -1,0 +1,67 @@
+"""Reusable call site for ``tilemix_prefill_fwd``: keeps a batch's device-side
+metadata (offsets, routing words, grouping factors) and the workspace, so a
+step only marshals the four tensor pointers."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (BLOCK_M, make_args, tilemix_prefill_fwd, tilemix_tile_offsets,
+               tilemix_workspace_size)
+
+
+class TileMixPrefill:
+    def __init__(self, lengths, hq, hk, d, masks, g, causal=True, softmax_scale=0.0,
+                 kv_head_of_q=None, device="cuda"):
+        self.lengths = [int(x) for x in lengths]
+        self.hq, self.hk, self.d = int(hq), int(hk), int(d)
+        cu = np.zeros(len(self.lengths) + 1, dtype=np.int32)
+        cu[1:] = np.cumsum(self.lengths)
+        cq, ck = tilemix_tile_offsets(cu)
+        self.nseq = len(self.lengths)
+        self.total_tokens = int(cu[-1])
+        self.total_qtiles = int(cq[-1])
+        self.total_ktiles = int(ck[-1])
+        self.max_seqlen = max(self.lengths) if self.lengths else 0
+        self.causal = bool(causal)
+        self.softmax_scale = float(softmax_scale)
+        self.device = torch.device(device)
+        masks = np.ascontiguousarray(masks, dtype=np.uint64)
+        if masks.shape != (self.total_qtiles, self.hk):
+            raise ValueError("masks must be [total_qtiles, hk] = [%d, %d]"
+                             % (self.total_qtiles, self.hk))
+        self.cu_seqlens = torch.from_numpy(cu).to(self.device)
+        self.cu_qtiles = torch.from_numpy(cq).to(self.device)
+        self.cu_ktiles = torch.from_numpy(ck).to(self.device)
+        self.masks = torch.from_numpy(masks.view(np.int64)).to(self.device)
+        self.g = torch.as_tensor(np.asarray(g, dtype=np.int32)).to(self.device)
+        self.kv_head_of_q = (None if kv_head_of_q is None else
+                             torch.as_tensor(np.asarray(kv_head_of_q, dtype=np.int32)).to(self.device))
+        self.workspace = None
+
+    @property
+    def max_qtiles(self):
+        return (self.max_seqlen + BLOCK_M - 1) // BLOCK_M
+
+    def args(self, q, k, v, o, lse=None, k_i8=None, k_scale=None, debug_int32_scores=None,
+             events=None):
+        return make_args(q, k, v, o, self.cu_seqlens, self.cu_qtiles, self.cu_ktiles, self.nseq,
+                         self.total_tokens, self.total_qtiles, self.total_ktiles,
+                         self.max_seqlen, self.masks, self.g, causal=self.causal,
+                         softmax_scale=self.softmax_scale, kv_head_of_q=self.kv_head_of_q,
+                         lse=lse, k_i8=k_i8, k_scale=k_scale, workspace=self.workspace,
+                         debug_int32_scores=debug_int32_scores, events=events)
+
+    def ensure_workspace(self, q, k, v, o, **kw):
+        a = self.args(q, k, v, o, **kw)
+        need = tilemix_workspace_size(a)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        return self.workspace
+
+    def __call__(self, q, k, v, o=None, lse=None, stream=None, **kw):
+        if o is None:
+            o = torch.empty_like(q)
+        self.ensure_workspace(q, k, v, o, lse=lse, **kw)
+        tilemix_prefill_fwd(self.args(q, k, v, o, lse=lse, **kw), stream)
+        return o
