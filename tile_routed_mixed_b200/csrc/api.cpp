@@ -223,7 +223,7 @@ TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream)
   p.total_tokens = T;
   p.total_qtiles = a->total_qtiles;
   p.total_ktiles = a->total_ktiles;
-  p.max_qtiles = (a->max_seqlen + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M;
+  p.max_qpairs = ((a->max_seqlen + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M + 1) / 2;
   p.hq = a->hq;
   p.hk = a->hk;
   p.group = a->hq / a->hk;

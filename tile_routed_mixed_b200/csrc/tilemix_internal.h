@@ -35,7 +35,7 @@ struct PrefillParams {
   const float* k_scale;   // [hk][total_ktiles]
   int32_t* dbg;
   int dbg_cols;
-  int nseq, total_tokens, total_qtiles, total_ktiles, max_qtiles;
+  int nseq, total_tokens, total_qtiles, total_ktiles, max_qpairs;
   int hq, hk, group;      // group = hq / hk
   int causal;
   float scale_log2;       // softmax scale * log2(e)

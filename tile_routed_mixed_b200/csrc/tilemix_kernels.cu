@@ -23,6 +23,22 @@ namespace tilemix {
 // tilemix_get_error().
 __device__ unsigned int g_status;
 
+#ifdef TILEMIX_TRACE
+// Profiling builds only: SM clock stamps of pipeline events of one CTA,
+// trace[(event * 2 + q) * 256 + tile].
+__device__ unsigned long long* g_trace;
+__device__ int g_trace_cta;
+#define TRACE(ev, q, i)                                                              \
+  do {                                                                               \
+    if (g_trace && static_cast<int>(blockIdx.x) == g_trace_cta && (i) < 256)         \
+      g_trace[((ev) * 2 + (q)) * 256 + (i)] = clock64();                             \
+  } while (0)
+#else
+#define TRACE(ev, q, i) \
+  do {                  \
+  } while (0)
+#endif
+
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 64;   // keys per tile
 
@@ -116,56 +132,83 @@ int launch_quantize(const void* x, const int32_t* cu_seqlens, const int32_t* cu_
 // ===================================================================
 // Fused attention forward.
 //
-// One CTA per (query-tile row, query head), heaviest rows first.  Warp roles:
-//   warp 0     TMA producer: Q (fp16 + int8), then per key tile either the
-//              fp16 or the int8 K tile (by the routing bit) and the fp16 V tile
-//   warp 1     TMEM owner and MMA issuer: S = Q K^T (kind::f16 -> f32 or
-//              kind::i8 -> s32) into one of two TMEM score buffers, then
-//              O += P V (kind::f16, P read from TMEM)
-//   warps 4-7  softmax: one query row per thread; routed scores -> float
-//              score domain, legality mask, online max / normaliser, P in
-//              fp16 back to TMEM; final O / l in fp16
+// One CTA per (sequence, query head, pair of query-tile rows 2j and 2j+1),
+// heaviest pairs first.  The two 128-row Q tiles share every K/V tile load.
+// Warp roles (16 warps, four warpgroups):
+//   warp 0      TMA producer: both Q tiles (fp16 and int8), then per key tile
+//               the K tile in each precision the two rows' routing bits need,
+//               and the fp16 V tile
+//   warps 1, 2  MMA issuers of Q tile 0 and Q tile 1 (warp 1 also owns TMEM):
+//               S_q = Q_q K^T (kind::f16 -> f32 or kind::i8 -> s32, by row
+//               q's routing bit) into one of the two TMEM score buffers of Q
+//               tile q, then O_q += P_q V (kind::f16, P read from TMEM)
+//   warps 4-7   softmax of Q tile 0, warps 8-11 softmax of Q tile 1: one query
+//               row per thread; routed scores -> float score domain, legality
+//               mask, online max / normaliser, P in fp16 back to TMEM; at the
+//               end O / l in fp16
+//   warps 12-15 correction of Q tile 0, warps 16-19 of Q tile 1: when a row's
+//               running max moved, rescale its O accumulator in TMEM (after
+//               the previous P.V landed) before the next P.V is issued, off
+//               the softmax warps' critical path
+// TMEM (512 columns): per Q tile q, O_q [D cols] and two 64-column score
+// buffers, at column offset 256 q.
 // ===================================================================
 constexpr int kStages = 3;
-constexpr int kPrefillThreads = 256;
+constexpr int kPrefillThreads = 640;
+constexpr int kCorrectionWarp0 = 12;
+// Register split (setmaxnreg): producer/MMA warpgroup, two softmax
+// warpgroups, two correction warpgroups.  128 * (64 + 2 * 152 + 2 * 48) =
+// 59392 <= 640 threads * 96 registers at launch.
+constexpr uint32_t kRegsControl = 64;
+constexpr uint32_t kRegsSoftmax = 152;
+constexpr uint32_t kRegsCorrection = 48;
 constexpr int kSoftmaxWarp0 = 4;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
-constexpr uint32_t kTmemCols = 256;
+// Lazy rescaling: the running max used for P is only moved when the tile max
+// exceeds it by more than this (log2 units), so P <= 2^15 stays inside fp16
+// (65504) and P.V / the normaliser stay exact in their fp32 accumulators.  A
+// stale max only shifts fp16 underflow further below the true maximum.
+constexpr float kRescaleThreshold = 15.0f;
+constexpr uint32_t kTmemCols = 512;
 
 template <int D>
 struct Smem {
   static constexpr int kQ = BM * D * 2;       // fp16 Q tile
   static constexpr int kQ8 = BM * D;          // int8 Q tile
-  static constexpr int kKSlot = BN * D * 2;   // fp16 K tile (an int8 K tile uses half)
+  static constexpr int kK16 = BN * D * 2;     // fp16 K tile
+  static constexpr int kK8 = BN * D;          // int8 K tile
   static constexpr int kV = BN * D * 2;       // fp16 V tile
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffQ8 = kOffQ + kQ;
-  static constexpr int kOffK = kOffQ8 + kQ8;
-  static constexpr int kOffV = kOffK + kStages * kKSlot;
+  static constexpr int kOffQ = 0;                          // + q * kQ
+  static constexpr int kOffQ8 = kOffQ + 2 * kQ;            // + q * kQ8
+  static constexpr int kOffK16 = kOffQ8 + 2 * kQ8;         // + stage * kK16
+  static constexpr int kOffK8 = kOffK16 + kStages * kK16;  // + stage * kK8
+  static constexpr int kOffV = kOffK8 + kStages * kK8;     // + stage * kV
   static constexpr int kOffBar = kOffV + kStages * kV;
-  static constexpr int kBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
+  static constexpr int kOffAlpha = kOffBar + 512;          // float [2][2][128]
+  static constexpr int kBytes = kOffAlpha + 2048 + 1024;    // + alignment slack
   static constexpr int kF16Steps = D / 16;
   static constexpr int kI8Steps = D / 32;
   static constexpr uint32_t kI8Layout = D == 128 ? ptx::kSwizzle128B : ptx::kSwizzle64B;
   static constexpr uint32_t kI8Sbo = 8 * D;  // 8 rows of D bytes
-  static constexpr uint32_t kColO = 0;
-  static constexpr uint32_t kColS = D;       // two 64-column score buffers
+  __host__ __device__ static constexpr uint32_t col_o(int q) { return 256u * q; }
+  __host__ __device__ static constexpr uint32_t col_s(int q, int b) { return 256u * q + D + 64u * b; }
 };
 
 // Every mbarrier below is waited on by parity.  A parity wait is only
 // unambiguous when the waiter is at most one phase behind the barrier, so each
-// barrier is sized so that this holds: e.g. P(j).V completions alternate
-// between two barriers (at tile i the softmax waits for P(i-1).V, and
-// P(i-3).V is already known complete because S(i-1) could only be computed
-// after it), and the epilogue waits on a barrier of its own.
+// barrier is sized so that this holds: e.g. the P.V completions of a Q tile
+// alternate between two barriers (at key tile i its softmax waits for
+// P(i-1).V, and P(i-3).V is already known complete because the commit that
+// signalled S(i-1) covers every MMA issued before it), and the epilogue waits
+// on a barrier of its own.
 struct Barriers {
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2];
-  uint64_t pv_done[2];  // P(j).V of tile j done, one barrier per score buffer
-  uint64_t o_final;     // the last P.V of the CTA done
-  uint64_t drain;
+  uint64_t kv_full[kStages];   // K (both precisions needed) and V of a key tile landed
+  uint64_t kv_empty[kStages];  // P.V of that key tile done by every Q tile using it
+  uint64_t s_full[2][2], p_full[2][2];  // [Q tile][score buffer]
+  uint64_t pv_done[2][2];               // P(j).V of Q tile q done, buffer j & 1
+  uint64_t o_ready[2][2];               // O_q rescaled (if needed) for P(j).V
+  uint64_t o_final[2];                  // the last P.V of Q tile q done
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -210,9 +253,85 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity,
   }
 }
 
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ bool routed_int8(uint64_t word, int kt, int g) {
   return (word >> (kt / g)) & 1ull;
 }
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+
+// s += low half + high half of a packed f16x2 (each widened exactly).
+__device__ __forceinline__ void add_f16x2_to_f32(float& s, uint32_t h2) {
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+      : "+f"(s)
+      : "r"(h2));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Shared-memory descriptor from a template holding every field but the start
+// address.
+__device__ __forceinline__ uint64_t desc_at(uint64_t tmpl, uint32_t addr) {
+  return tmpl | static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+}
+
+// S = Q K^T of one 128 x 64 score tile into TMEM column d_s, in the precision
+// the routing bit selects.
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_s, bool is_int, uint32_t aq16, uint32_t aq8,
+                                         uint32_t bk16, uint32_t bk8, uint64_t tmpl16,
+                                         uint64_t tmpl8) {
+  constexpr uint32_t kIdF16 = ptx::idesc_f16(BM, BN, false);
+  constexpr uint32_t kIdI8 = ptx::idesc_s8(BM, BN);
+  if (is_int) {
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k)
+      ptx::mma_i8_ss(d_s, desc_at(tmpl8, aq8 + k * 32), desc_at(tmpl8, bk8 + k * 32), kIdI8,
+                     k > 0 ? 1u : 0u);
+  } else {
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k)
+      ptx::mma_f16_ss(d_s, desc_at(tmpl16, aq16 + (k >> 2) * (BM * 128) + (k & 3) * 32),
+                      desc_at(tmpl16, bk16 + (k >> 2) * (BN * 128) + (k & 3) * 32), kIdF16,
+                      k > 0 ? 1u : 0u);
+  }
+}
+
+// O += P V of one 64-key tile: P (fp16) from TMEM column a_p, V from shared
+// memory (MN-major).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint32_t vbase,
+                                         uint64_t tmplv, bool first) {
+  constexpr uint32_t kIdPV = ptx::idesc_f16(BM, D, true);
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    ptx::mma_f16_ts(d_o, a_p + kk * 8, desc_at(tmplv, vbase + kk * 2048), kIdPV,
+                    (!first || kk > 0) ? 1u : 0u);
+}
+
+// Per-Q-tile geometry of a CTA.
+struct QTile {
+  int qt;        // query-tile row inside the sequence
+  int row0;      // first query row
+  int ntiles;    // legal key tiles (0 if this Q tile does not exist)
+  uint64_t word; // routing word of (row, KV head)
+};
 
 template <int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -226,27 +345,42 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   // A wait of an earlier CTA already expired: do not start more work.
   if (*reinterpret_cast<volatile unsigned int*>(&g_status) & kStatusTimeout) return;
 
-  // ---- work item: heaviest query-tile rows first ----
+  // ---- work item: heaviest query-tile pairs first, heads innermost ----
   int b = blockIdx.x;
   const int h = b % p.hq;
   b /= p.hq;
   const int s = b % p.nseq;
   b /= p.nseq;
-  const int qt = p.max_qtiles - 1 - b;
+  const int pair = p.max_qpairs - 1 - b;
   const int t0 = p.cu_seqlens[s];
   const int L = p.cu_seqlens[s + 1] - t0;
-  if (qt >= (L + BM - 1) / BM) return;
+  const int tm = (L + BM - 1) / BM;
+  if (2 * pair >= tm) return;
   const int kv = p.kv_head_of_q ? p.kv_head_of_q[h] : h / p.group;
-  const int row0 = qt * BM;
-  // causal and boundary legality: independent of the routing word
-  const int last_tile = p.causal ? (min(row0 + BM, L) - 1) / BN : (L - 1) / BN;
-  const int ntiles = last_tile + 1;
   const int gs = p.g[s];
-  if (gs < 1 || last_tile / gs > 63) {
+  QTile qtile[2];
+  int nt = 0;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    QTile& t = qtile[q];
+    t.qt = 2 * pair + q;
+    t.row0 = t.qt * BM;
+    if (t.qt < tm) {
+      // causal and boundary legality: independent of the routing word
+      const int last = p.causal ? (min(t.row0 + BM, L) - 1) / BN : (L - 1) / BN;
+      t.ntiles = last + 1;
+      t.word = p.masks[static_cast<size_t>(p.cu_qtiles[s] + t.qt) * p.hk + kv];
+    } else {
+      t.ntiles = 0;
+      t.word = 0;
+    }
+    nt = max(nt, t.ntiles);
+  }
+  if (gs < 1 || (nt - 1) / gs > 63) {
     if (threadIdx.x == 0) atomicOr(&g_status, kStatusBadGroups);
     return;
   }
-  const uint64_t word = p.masks[static_cast<size_t>(p.cu_qtiles[s] + qt) * p.hk + kv];
+  const int nq = qtile[1].ntiles > 0 ? 2 : 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -254,19 +388,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->q_full, 1);
     for (int i = 0; i < kStages; ++i) {
-      ptx::mbar_init(&bars->k_full[i], 1);
-      ptx::mbar_init(&bars->k_empty[i], 1);
-      ptx::mbar_init(&bars->v_full[i], 1);
-      ptx::mbar_init(&bars->v_empty[i], 1);
+      ptx::mbar_init(&bars->kv_full[i], 1);
+      ptx::mbar_init(&bars->kv_empty[i], nq);
     }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&bars->s_full[i], 1);
-      ptx::mbar_init(&bars->p_full[i], 128);
+    for (int q = 0; q < 2; ++q) {
+      for (int i = 0; i < 2; ++i) {
+        ptx::mbar_init(&bars->s_full[q][i], 1);
+        ptx::mbar_init(&bars->p_full[q][i], 128);
+        ptx::mbar_init(&bars->pv_done[q][i], 1);
+        ptx::mbar_init(&bars->o_ready[q][i], 128);
+      }
+      ptx::mbar_init(&bars->o_final[q], 1);
     }
-    ptx::mbar_init(&bars->pv_done[0], 1);
-    ptx::mbar_init(&bars->pv_done[1], 1);
-    ptx::mbar_init(&bars->o_final, 1);
-    ptx::mbar_init(&bars->drain, 1);
+    ptx::mbar_init(&bars->drain[0], 1);
+    ptx::mbar_init(&bars->drain[1], 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -281,252 +416,316 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   volatile int* abort_flag = &bars->abort;
   const unsigned long long tmo = p.timeout_ns;
 
-  uint8_t* sQ = smem + S::kOffQ;
-  uint8_t* sQ8 = smem + S::kOffQ8;
-  uint8_t* sK = smem + S::kOffK;
-  uint8_t* sV = smem + S::kOffV;
+  float* alpha_smem = reinterpret_cast<float*>(smem + S::kOffAlpha);  // [q][buffer][row]
 
+  if (warp < 4) {
+    regs_dec<kRegsControl>();
+  }
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
-      ptx::prefetch_tensormap(&p.tm_q);
       ptx::prefetch_tensormap(&p.tm_k);
+      ptx::prefetch_tensormap(&p.tm_k8);
       ptx::prefetch_tensormap(&p.tm_v);
-      ptx::mbar_expect_tx(&bars->q_full, S::kQ + S::kQ8);
-#pragma unroll
-      for (int j = 0; j < D / 64; ++j)
-        ptx::tma_load_3d(sQ + j * BM * 128, &p.tm_q, &bars->q_full, j * 64, h, t0 + row0);
-      ptx::tma_load_3d(sQ8, &p.tm_q8, &bars->q_full, 0, h, t0 + row0);
-      int kcnt[kStages] = {}, vcnt[kStages] = {};
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i % kStages;
-        const uint32_t ph = ((i / kStages) - 1) & 1;
-        if (i >= kStages && !wait_bar(&bars->k_empty[st], ph, abort_flag, tmo)) break;
-        const int key0 = t0 + i * BN;
-        uint8_t* kslot = sK + st * S::kKSlot;
-        if (routed_int8(word, i, gs)) {
-          ptx::mbar_expect_tx(&bars->k_full[st], BN * D);
-          ptx::tma_load_3d(kslot, &p.tm_k8, &bars->k_full[st], 0, kv, key0);
-        } else {
-          ptx::mbar_expect_tx(&bars->k_full[st], BN * D * 2);
-#pragma unroll
-          for (int j = 0; j < D / 64; ++j)
-            ptx::tma_load_3d(kslot + j * BN * 128, &p.tm_k, &bars->k_full[st], j * 64, kv, key0);
-        }
-        ++kcnt[st];
-        if (i >= kStages && !wait_bar(&bars->v_empty[st], ph, abort_flag, tmo)) break;
-        uint8_t* vslot = sV + st * S::kV;
-        ptx::mbar_expect_tx(&bars->v_full[st], BN * D * 2);
+      ptx::mbar_expect_tx(&bars->q_full, nq * (S::kQ + S::kQ8));
+      for (int q = 0; q < nq; ++q) {
 #pragma unroll
         for (int j = 0; j < D / 64; ++j)
-          ptx::tma_load_3d(vslot + j * BN * 128, &p.tm_v, &bars->v_full[st], j * 64, kv, key0);
-        ++vcnt[st];
+          ptx::tma_load_3d(smem + S::kOffQ + q * S::kQ + j * BM * 128, &p.tm_q, &bars->q_full,
+                           j * 64, h, t0 + qtile[q].row0);
+        ptx::tma_load_3d(smem + S::kOffQ8 + q * S::kQ8, &p.tm_q8, &bars->q_full, 0, h,
+                         t0 + qtile[q].row0);
+      }
+      int cnt[kStages] = {};
+      for (int i = 0; i < nt; ++i) {
+        const int st = i % kStages;
+        bool need16 = false, need8 = false;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          if (i < qtile[q].ntiles) {
+            if (routed_int8(qtile[q].word, i, gs)) need8 = true;
+            else need16 = true;
+          }
+        }
+        if (i >= kStages && !wait_bar(&bars->kv_empty[st], ((i / kStages) - 1) & 1, abort_flag, tmo))
+          break;
+        const int key0 = t0 + i * BN;
+        uint64_t* full = &bars->kv_full[st];
+        ptx::mbar_expect_tx(full, (need16 ? S::kK16 : 0) + (need8 ? S::kK8 : 0) + S::kV);
+        if (need16) {
+#pragma unroll
+          for (int j = 0; j < D / 64; ++j)
+            ptx::tma_load_3d(smem + S::kOffK16 + st * S::kK16 + j * BN * 128, &p.tm_k, full,
+                             j * 64, kv, key0);
+        }
+        if (need8)
+          ptx::tma_load_3d(smem + S::kOffK8 + st * S::kK8, &p.tm_k8, full, 0, kv, key0);
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j)
+          ptx::tma_load_3d(smem + S::kOffV + st * S::kV + j * BN * 128, &p.tm_v, full, j * 64, kv,
+                           key0);
+        ++cnt[st];
       }
       // Never leave with copies into this CTA's shared memory in flight.
       drain_bar(&bars->q_full, 0, tmo);
-      for (int st = 0; st < kStages; ++st) {
-        if (kcnt[st]) drain_bar(&bars->k_full[st], (kcnt[st] - 1) & 1, tmo);
-        if (vcnt[st]) drain_bar(&bars->v_full[st], (vcnt[st] - 1) & 1, tmo);
-      }
+      for (int st = 0; st < kStages; ++st)
+        if (cnt[st]) drain_bar(&bars->kv_full[st], (cnt[st] - 1) & 1, tmo);
     }
-  } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
-      constexpr uint32_t kIdF16 = ptx::idesc_f16(BM, BN, false);
-      constexpr uint32_t kIdI8 = ptx::idesc_s8(BM, BN);
-      constexpr uint32_t kIdPV = ptx::idesc_f16(BM, D, true);
-      const uint32_t aQ = ptx::smem_addr(sQ), aQ8 = ptx::smem_addr(sQ8);
-      const uint32_t aK = ptx::smem_addr(sK), aV = ptx::smem_addr(sV);
+  } else if (warp == 1 || warp == 2) {
+    // ================= MMA issuers: warp 1 for Q tile 0, warp 2 for Q tile 1 =====
+    // Order: S_q(0), S_q(1), then per key tile j: P_q(j).V followed at once by
+    // S_q(j + 2), which reuses the score buffer P_q(j) was read from:
+    // tcgen05.mma operations of one thread run in issue order, so no wait is
+    // needed for that reuse.  A thread whose Q tile is shorter (or absent) still releases
+    // the remaining K/V stages, after they are loaded, so that each stage's
+    // release barrier sees one arrival per Q tile.
+    const int q = warp - 1;
+    if (lane == 0 && q < nq) {
+      const uint32_t a_smem = ptx::smem_addr(smem);
+      const uint64_t t16 = ptx::smem_desc(0, 16, 1024, ptx::kSwizzle128B);
+      const uint64_t t8 = ptx::smem_desc(0, 16, S::kI8Sbo, S::kI8Layout);
+      const uint64_t tv = ptx::smem_desc(0, BN * 128, 1024, ptx::kSwizzle128B);
+      const int ntq = qtile[q].ntiles;
+      const uint64_t word = qtile[q].word;
+      const uint32_t aq16 = a_smem + S::kOffQ + q * S::kQ;
+      const uint32_t aq8 = a_smem + S::kOffQ8 + q * S::kQ8;
+      const uint32_t d_o = tmem + S::col_o(q);
       bool ok = wait_bar(&bars->q_full, 0, abort_flag, tmo);
       ptx::tc_fence_after();
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j % kStages;
-        const int sb = j & 1;
-        if (!wait_bar(&bars->p_full[sb], (j >> 1) & 1, abort_flag, tmo)) return false;
-        if (!wait_bar(&bars->v_full[st], (j / kStages) & 1, abort_flag, tmo)) return false;
-        ptx::tc_fence_after();
-        const int valid = L - j * BN;
-        if (valid < BN) {
-          // Keys past the sequence end belong to the next packed sequence:
-          // zero their V rows so that 0 * (NaN or Inf) cannot reach O.
-          uint8_t* vslot = sV + st * S::kV;
-          for (int part = 0; part < D / 64; ++part)
-            for (int r = valid; r < BN; ++r) {
-              uint4* row = reinterpret_cast<uint4*>(vslot + part * BN * 128 + r * 128);
-#pragma unroll
-              for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
-            }
-          ptx::fence_proxy_async_smem();
-        }
-        const uint32_t vbase = aV + st * S::kV;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc = ptx::smem_desc(vbase + kk * 2048, BN * 128, 1024, ptx::kSwizzle128B);
-          ptx::mma_f16_ts(tmem + S::kColO, tmem + S::kColS + sb * 64 + kk * 8, bdesc, kIdPV,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        ptx::mma_commit(&bars->pv_done[sb]);
-        ptx::mma_commit(&bars->v_empty[st]);
-        if (j == ntiles - 1) ptx::mma_commit(&bars->o_final);
-        return true;
-      };
-      for (int i = 0; ok && i < ntiles; ++i) {
+      // S(i) for the first two tiles; afterwards S(j + 2) follows P(j).V at once
+      // so that the score buffer is refilled as early as possible.
+      for (int i = 0; ok && i < 2 && i < ntq; ++i) {
         const int st = i % kStages;
-        const int sb = i & 1;
-        // score buffer sb is free once P(i-2).V has read P(i-2) from it
-        if (i >= 2 && !wait_bar(&bars->pv_done[sb], ((i - 2) >> 1) & 1, abort_flag, tmo)) {
+        if (!wait_bar(&bars->kv_full[st], (i / kStages) & 1, abort_flag, tmo)) {
           ok = false;
           break;
         }
-        if (!wait_bar(&bars->k_full[st], (i / kStages) & 1, abort_flag, tmo)) { ok = false; break; }
         ptx::tc_fence_after();
-        const uint32_t d_s = tmem + S::kColS + sb * 64;
-        const uint32_t kbase = aK + st * S::kKSlot;
-        if (routed_int8(word, i, gs)) {
+        issue_qk<D>(tmem + S::col_s(q, i & 1), routed_int8(word, i, gs), aq16, aq8,
+                    a_smem + S::kOffK16 + st * S::kK16, a_smem + S::kOffK8 + st * S::kK8, t16,
+                    t8);
+        ptx::mma_commit(&bars->s_full[q][i & 1]);
+        TRACE(4, q, i);
+      }
+      for (int j = 0; ok && j < nt; ++j) {
+        const int st = j % kStages;
+        if (j < ntq) {
+          const int sb = j & 1;
+          const int valid = L - j * BN;
+          if (valid < BN) {
+            // Keys past the sequence end belong to the next packed sequence:
+            // zero their V rows so that 0 * (NaN or Inf) cannot reach O.  The
+            // Q tiles write the same zeros, each before its own P.V.
+            uint8_t* vslot = smem + S::kOffV + st * S::kV;
+            for (int part = 0; part < D / 64; ++part)
+              for (int r = valid; r < BN; ++r) {
+                uint4* row = reinterpret_cast<uint4*>(vslot + part * BN * 128 + r * 128);
 #pragma unroll
-          for (int k = 0; k < S::kI8Steps; ++k) {
-            const uint64_t ad = ptx::smem_desc(aQ8 + k * 32, 16, S::kI8Sbo, S::kI8Layout);
-            const uint64_t bd = ptx::smem_desc(kbase + k * 32, 16, S::kI8Sbo, S::kI8Layout);
-            ptx::mma_i8_ss(d_s, ad, bd, kIdI8, k > 0 ? 1u : 0u);
+                for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+              }
+            ptx::fence_proxy_async_smem();
           }
+          if (!wait_bar(&bars->o_ready[q][sb], (j >> 1) & 1, abort_flag, tmo)) {
+            ok = false;
+            break;
+          }
+          TRACE(10, q, j);
+          ptx::tc_fence_after();
+          issue_pv<D>(d_o, tmem + S::col_s(q, sb), a_smem + S::kOffV + st * S::kV, tv, j == 0);
+          TRACE(5, q, j);
+          const int i = j + 2;
+          if (i < ntq) {
+            const int sti = i % kStages;
+            if (!wait_bar(&bars->kv_full[sti], (i / kStages) & 1, abort_flag, tmo)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            issue_qk<D>(tmem + S::col_s(q, sb), routed_int8(word, i, gs), aq16, aq8,
+                        a_smem + S::kOffK16 + sti * S::kK16, a_smem + S::kOffK8 + sti * S::kK8,
+                        t16, t8);
+            ptx::mma_commit(&bars->s_full[q][sb]);
+            TRACE(4, q, i);
+          }
+          ptx::mma_commit(&bars->pv_done[q][sb]);
+          if (j == ntq - 1) ptx::mma_commit(&bars->o_final[q]);
         } else {
-#pragma unroll
-          for (int k = 0; k < S::kF16Steps; ++k) {
-            const uint64_t ad = ptx::smem_desc(aQ + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024,
-                                               ptx::kSwizzle128B);
-            const uint64_t bd = ptx::smem_desc(kbase + (k >> 2) * (BN * 128) + (k & 3) * 32, 16,
-                                               1024, ptx::kSwizzle128B);
-            ptx::mma_f16_ss(d_s, ad, bd, kIdF16, k > 0 ? 1u : 0u);
+          // a tile this Q tile does not use: release it once it is loaded
+          if (!wait_bar(&bars->kv_full[st], (j / kStages) & 1, abort_flag, tmo)) {
+            ok = false;
+            break;
           }
         }
-        ptx::mma_commit(&bars->s_full[sb]);
-        ptx::mma_commit(&bars->k_empty[st]);
-        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+        ptx::mma_commit(&bars->kv_empty[st]);
       }
-      if (ok) issue_pv(ntiles - 1);
-      // all MMAs of this CTA complete before TMEM and shared memory go away
-      ptx::mma_commit(&bars->drain);
-      drain_bar(&bars->drain, 0, tmo);
+      // all MMAs of this thread complete before TMEM and shared memory go away
+      ptx::mma_commit(&bars->drain[q]);
+      drain_bar(&bars->drain[q], 0, tmo);
     }
-  } else if (warp >= kSoftmaxWarp0) {
+  } else if (warp >= kSoftmaxWarp0 && warp < kCorrectionWarp0) {
     // ================= softmax / epilogue =================
-    const int tr = threadIdx.x - kSoftmaxWarp0 * 32;  // row within the tile
-    const int wq = warp - kSoftmaxWarp0;              // TMEM lane quarter
-    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const int my_row = row0 + tr;
-    const float q_sc =
-        p.q_scale[static_cast<size_t>(h) * p.total_qtiles + p.cu_qtiles[s] + qt];
-    const float* ks = p.k_scale + static_cast<size_t>(kv) * p.total_ktiles + p.cu_ktiles[s];
-    float m = -INFINITY;  // running max, log2 units
-    float l = 0.f;        // normaliser (sum of the fp16-rounded P)
-    bool ok = true;
-    uint32_t r[32], r2[32];
-    for (int i = 0; i < ntiles; ++i) {
-      const int sb = i & 1;
-      if (!wait_bar_warp(&bars->s_full[sb], (i >> 1) & 1, abort_flag, tmo)) { ok = false; break; }
-      ptx::tc_fence_after();
-      const uint32_t ts = tmem + lane_base + S::kColS + sb * 64;
-      ptx::tmem_ld32(ts, r);
-      ptx::tmem_ld32(ts + 32, r2);
-      ptx::tmem_ld_wait();
-      const bool is_int = routed_int8(word, i, gs);
-      float x[64];
-      if (is_int) {
-        const float sc = q_sc * __ldg(ks + i) * p.scale_log2;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          x[j] = static_cast<float>(static_cast<int>(r[j])) * sc;
-          x[32 + j] = static_cast<float>(static_cast<int>(r2[j])) * sc;
-        }
-        if (p.dbg && my_row < L) {
-          int32_t* drow = p.dbg + (static_cast<size_t>(h) * p.total_tokens + t0 + my_row) * p.dbg_cols;
-          for (int j = 0; j < 64; ++j) {
-            const int key = i * BN + j;
-            if (key < L) drow[key] = static_cast<int32_t>(j < 32 ? r[j] : r2[j - 32]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          x[j] = __uint_as_float(r[j]) * p.scale_log2;
-          x[32 + j] = __uint_as_float(r2[j]) * p.scale_log2;
-        }
-      }
-      const int key0 = i * BN;
-      if (key0 + BN > L || (p.causal && key0 + BN - 1 > row0)) {
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int key = key0 + j;
-          if (key >= L || (p.causal && key > my_row)) x[j] = -INFINITY;
-        }
-      }
-      float tmax = x[0];
-#pragma unroll
-      for (int j = 1; j < 64; ++j) tmax = fmaxf(tmax, x[j]);
-      const float m_new = fmaxf(m, tmax);
-      const bool resc = m_new - m > kRescaleThreshold;
-      const float m_use = resc ? m_new : m;
-      const float alpha = resc ? ptx::ex2(m - m_new) : 1.0f;
-      float lsum = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const __half2 hp = __floats2half2_rn(ptx::ex2(x[2 * j] - m_use), ptx::ex2(x[2 * j + 1] - m_use));
-        const float2 back = __half22float2(hp);
-        lsum += back.x + back.y;
-        pk[j] = *reinterpret_cast<const uint32_t*>(&hp);
-      }
-      l = l * alpha + lsum;
-      m = m_use;
-      if (__any_sync(0xffffffffu, resc && i > 0)) {
-        // O holds P.V of tiles < i: rescale it once P(i-1).V has landed.
-        if (!wait_bar_warp(&bars->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, tmo)) {
+    regs_inc<kRegsSoftmax>();
+    const int q = (warp - kSoftmaxWarp0) >> 2;        // Q tile of this warpgroup
+    const int tr = threadIdx.x - (kSoftmaxWarp0 + 4 * q) * 32;  // row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const QTile t = qtile[q];
+    const int my_row = t.row0 + tr;
+    if (t.ntiles > 0) {
+      const float q_sc =
+          p.q_scale[static_cast<size_t>(h) * p.total_qtiles + p.cu_qtiles[s] + t.qt];
+      const float* ks = p.k_scale + static_cast<size_t>(kv) * p.total_ktiles + p.cu_ktiles[s];
+      float m = -INFINITY;  // running max, log2 units
+      float l = 0.f;        // normaliser: sum of the fp16-rounded P actually used in P.V
+      bool ok = true;
+      uint32_t r[64];
+      float k_sc_next = __ldg(ks);
+      for (int i = 0; i < t.ntiles; ++i) {
+        const int sb = i & 1;
+        const bool is_int = routed_int8(t.word, i, gs);
+        const float k_sc = k_sc_next;
+        if (i + 1 < t.ntiles) k_sc_next = __ldg(ks + i + 1);
+        if (!wait_bar_warp(&bars->s_full[q][sb], (i >> 1) & 1, abort_flag, tmo)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
+        if (tr == 0) TRACE(0, q, i);
+        const uint32_t ts = tmem + lane_base + S::col_s(q, sb);
+        ptx::tmem_ld32(ts, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        ptx::tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        ptx::tmem_ld_wait();
+        if (tr == 0) TRACE(11, q, i);
+        if (is_int && p.dbg && my_row < L) {
+          int32_t* drow =
+              p.dbg + (static_cast<size_t>(h) * p.total_tokens + t0 + my_row) * p.dbg_cols;
+          for (int j = 0; j < 64; ++j)
+            if (i * BN + j < L) drow[i * BN + j] = static_cast<int32_t>(r[j]);
+        }
+        // scores in the float domain, before the log2(e)-scaled softmax:
+        // FP16 tile: raw fp32 dot; INT8 tile: exact float of the INT32 dot.
+        if (is_int) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const uint32_t to = tmem + lane_base + S::kColO + c * 32;
+          for (int j = 0; j < 64; ++j) r[j] = __float_as_uint(__int2float_rn(static_cast<int>(r[j])));
+        }
+        const float c = is_int ? q_sc * k_sc * p.scale_log2 : p.scale_log2;
+        const int key0 = i * BN;
+        const bool masked = key0 + BN > L || (p.causal && key0 + BN - 1 > t.row0);
+        const int lim = p.causal ? min(L, my_row + 1) : L;  // legal keys < lim
+        if (masked) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            if (key0 + j >= lim) r[j] = __float_as_uint(-INFINITY);
+        }
+        // row max of the tile: eight independent chains, then a short tree
+        float g8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* x = reinterpret_cast<const float*>(&r[8 * u]);
+          g8[u] = fmaxf(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), x[6]), x[7]);
+        }
+        const float mx = fmaxf(max3(g8[0], g8[1], g8[2]), max3(max3(g8[3], g8[4], g8[5]), g8[6], g8[7]));
+        // c >= 0; c == 0 only for an all-zero quantisation block (scores 0)
+        const float m_tile = mx == -INFINITY ? -INFINITY : mx * c;
+        if (tr == 0) TRACE(12, q, i);
+        const float m_new = fmaxf(m, m_tile);
+        const bool resc = m_new - m > kRescaleThreshold;
+        const float m_use = resc ? m_new : m;
+        const float alpha = resc ? ptx::ex2(m - m_new) : 1.0f;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // P = 2^(score * c - m), packed in place: pair k lands in r[k]
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float x0 = fmaf(__uint_as_float(r[2 * k]), c, -m_use);
+          const float x1 = fmaf(__uint_as_float(r[2 * k + 1]), c, -m_use);
+          r[k] = pack_f16x2(ptx::ex2(x0), ptx::ex2(x1));
+          add_f16x2_to_f32(ls[k & 3], r[k]);
+        }
+        if (masked) {
+          // an all-zero block (c == 0) turns -inf scores into NaN: clear them
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const uint32_t keep = (key0 + 2 * k < lim ? 0x0000ffffu : 0u) |
+                                  (key0 + 2 * k + 1 < lim ? 0xffff0000u : 0u);
+            r[k] &= keep;
+          }
+          if (c == 0.f) {
+            ls[0] = ls[1] = ls[2] = ls[3] = 0.f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) add_f16x2_to_f32(ls[k & 3], r[k]);
+          }
+        }
+        l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        m = m_use;
+        if (tr == 0) TRACE(15, q, i);
+        // the correction warps rescale O by alpha before P(i).V is issued
+        alpha_smem[(q * 2 + sb) * BM + tr] = (i > 0) ? alpha : 1.0f;
+        ptx::tmem_st32(ts, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_full[q][sb]);
+        if (tr == 0) TRACE(1, q, i);
+      }
+      if (ok && wait_bar_warp(&bars->o_final[q], 0, abort_flag, tmo)) {
+        ptx::tc_fence_after();
+        const float inv_l = 1.0f / l;
+        const bool valid = my_row < L;
+        __half* orow = static_cast<__half*>(p.o) +
+                       (static_cast<size_t>(t0 + my_row) * p.hq + h) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          ptx::tmem_ld32(tmem + lane_base + S::col_o(q) + cc * 32,
+                         *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            r[32 + j] = pack_f16x2(__uint_as_float(r[2 * j]) * inv_l,
+                                   __uint_as_float(r[2 * j + 1]) * inv_l);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(r[32 + 4 * j], r[33 + 4 * j], r[34 + 4 * j], r[35 + 4 * j]);
+          }
+        }
+        if (p.lse && valid)
+          p.lse[static_cast<size_t>(h) * p.total_tokens + t0 + my_row] =
+              (m + __log2f(l)) * 0.69314718055994530942f;
+      }
+    }
+  } else if (warp >= kCorrectionWarp0) {
+    // ================= correction =================
+    regs_dec<kRegsCorrection>();
+    const int q = (warp - kCorrectionWarp0) >> 2;  // Q tile of this warpgroup
+    const int tr = threadIdx.x - (kCorrectionWarp0 + 4 * q) * 32;  // row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int ntq = qtile[q].ntiles;
+    uint32_t r[32];
+    for (int i = 0; i < ntq; ++i) {
+      const int sb = i & 1;
+      if (!wait_bar_warp(&bars->p_full[q][sb], (i >> 1) & 1, abort_flag, tmo)) break;
+      if (tr == 0) TRACE(2, q, i);
+      const float alpha = alpha_smem[(q * 2 + sb) * BM + tr];
+      if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+        // O_q holds P.V of tiles < i: rescale it once P(i-1).V has landed.
+        if (tr == 0) TRACE(13, q, i);
+        if (!wait_bar_warp(&bars->pv_done[q][(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, tmo))
+          break;
+        if (tr == 0) TRACE(14, q, i);
+        ptx::tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          const uint32_t to = tmem + lane_base + S::col_o(q) + cc * 32;
           ptx::tmem_ld32(to, r);
           ptx::tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
           ptx::tmem_st32(to, r);
         }
+        ptx::tmem_st_wait();
       }
-      ptx::tmem_st32(ts, pk);
-      ptx::tmem_st_wait();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->p_full[sb]);
-    }
-    if (ok && wait_bar_warp(&bars->o_final, 0, abort_flag, tmo)) {
-      ptx::tc_fence_after();
-      const float inv_l = 1.0f / l;
-      const bool valid = my_row < L;
-      __half* orow = static_cast<__half*>(p.o) +
-                     (static_cast<size_t>(t0 + my_row) * p.hq + h) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        ptx::tmem_ld32(tmem + lane_base + S::kColO + c * 32, r);
-        ptx::tmem_ld_wait();
-        uint32_t hv[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const __half2 o2 = __floats2half2_rn(__uint_as_float(r[2 * j]) * inv_l,
-                                               __uint_as_float(r[2 * j + 1]) * inv_l);
-          hv[j] = *reinterpret_cast<const uint32_t*>(&o2);
-        }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
-        }
-      }
-      if (p.lse && valid)
-        p.lse[static_cast<size_t>(h) * p.total_tokens + t0 + my_row] =
-            (m + __log2f(l)) * 0.69314718055994530942f;
+      ptx::mbar_arrive(&bars->o_ready[q][sb]);
+      if (tr == 0) TRACE(3, q, i);
     }
   }
 
@@ -544,7 +743,7 @@ static int launch_prefill_d(const PrefillParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return static_cast<int>(e);
-  const long long blocks = static_cast<long long>(p.max_qtiles) * p.nseq * p.hq;
+  const long long blocks = static_cast<long long>(p.max_qpairs) * p.nseq * p.hq;
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   prefill_fwd_kernel<D><<<static_cast<unsigned>(blocks), kPrefillThreads, smem, stream>>>(p);
@@ -556,6 +755,14 @@ int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream) {
   if (d == 64) return launch_prefill_d<64>(p, stream);
   return cudaErrorInvalidValue;
 }
+
+#ifdef TILEMIX_TRACE
+extern "C" TILEMIX_API int tilemix_trace_setup(void* buf, int cta) {
+  unsigned long long* ptr = static_cast<unsigned long long*>(buf);
+  if (cudaMemcpyToSymbol(g_trace, &ptr, sizeof(ptr)) != cudaSuccess) return 1;
+  return cudaMemcpyToSymbol(g_trace_cta, &cta, sizeof(cta)) != cudaSuccess;
+}
+#endif
 
 int read_and_clear_status(unsigned int* status, cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
