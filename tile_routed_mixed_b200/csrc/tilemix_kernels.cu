@@ -28,10 +28,9 @@ __device__ unsigned int g_status;
 // trace[(event * 2 + q) * 256 + tile].
 __device__ unsigned long long* g_trace;
 __device__ int g_trace_cta;
-#define TRACE(ev, q, i)                                                              \
-  do {                                                                               \
-    if (g_trace && static_cast<int>(blockIdx.x) == g_trace_cta && (i) < 256)         \
-      g_trace[((ev) * 2 + (q)) * 256 + (i)] = clock64();                             \
+#define TRACE(ev, q, i)                                               \
+  do {                                                                \
+    if (trace_buf && (i) < 256) trace_buf[((ev) * 2 + (q)) * 256 + (i)] = clock64(); \
   } while (0)
 #else
 #define TRACE(ev, q, i) \
@@ -157,9 +156,9 @@ constexpr int kStages = 3;
 constexpr int kPrefillThreads = 640;
 constexpr int kCorrectionWarp0 = 12;
 // Register split (setmaxnreg): producer/MMA warpgroup, two softmax
-// warpgroups, two correction warpgroups.  128 * (64 + 2 * 152 + 2 * 48) =
-// 59392 <= 640 threads * 96 registers at launch.
-constexpr uint32_t kRegsControl = 64;
+// warpgroups, two correction warpgroups.  128 * (80 + 2 * 152 + 2 * 48) =
+// 61440 = 640 threads * 96 registers at launch.
+constexpr uint32_t kRegsControl = 80;
 constexpr uint32_t kRegsSoftmax = 152;
 constexpr uint32_t kRegsCorrection = 48;
 constexpr int kSoftmaxWarp0 = 4;
@@ -189,22 +188,28 @@ struct Smem {
   static constexpr int kI8Steps = D / 32;
   static constexpr uint32_t kI8Layout = D == 128 ? ptx::kSwizzle128B : ptx::kSwizzle64B;
   static constexpr uint32_t kI8Sbo = 8 * D;  // 8 rows of D bytes
+  // TMEM columns of Q tile q: O [D], S [64], P buffers 0 and 1 [32 each]
   __host__ __device__ static constexpr uint32_t col_o(int q) { return 256u * q; }
-  __host__ __device__ static constexpr uint32_t col_s(int q, int b) { return 256u * q + D + 64u * b; }
+  __host__ __device__ static constexpr uint32_t col_s(int q) { return 256u * q + D; }
+  __host__ __device__ static constexpr uint32_t col_p(int q, int b) {
+    return 256u * q + D + 64u + 32u * b;
+  }
 };
 
 // Every mbarrier below is waited on by parity.  A parity wait is only
 // unambiguous when the waiter is at most one phase behind the barrier, so each
-// barrier is sized so that this holds: e.g. the P.V completions of a Q tile
-// alternate between two barriers (at key tile i its softmax waits for
-// P(i-1).V, and P(i-3).V is already known complete because the commit that
-// signalled S(i-1) covers every MMA issued before it), and the epilogue waits
-// on a barrier of its own.
+// barrier is sized so that this holds.  S is single-buffered: S(i+1) needs
+// s_free(i), which needs the softmax to have read S(i).  P is double-buffered
+// and the softmax stores P(i) only after P(i-2).V completed, so the
+// correction cannot fall two phases behind p_full, and every waiter of
+// pv_done / o_ready is at most one phase behind.
 struct Barriers {
   uint64_t q_full;
   uint64_t kv_full[kStages];   // K (both precisions needed) and V of a key tile landed
   uint64_t kv_empty[kStages];  // P.V of that key tile done by every Q tile using it
-  uint64_t s_full[2][2], p_full[2][2];  // [Q tile][score buffer]
+  uint64_t s_full[2];                   // S_q(i) in TMEM
+  uint64_t s_free[2];                   // S_q(i) read out: the S columns may be refilled
+  uint64_t p_full[2][2];                // P_q(j) in TMEM buffer j & 1
   uint64_t pv_done[2][2];               // P(j).V of Q tile q done, buffer j & 1
   uint64_t o_ready[2][2];               // O_q rescaled (if needed) for P(j).V
   uint64_t o_final[2];                  // the last P.V of Q tile q done
@@ -342,6 +347,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + S::kOffBar);
 
+#ifdef TILEMIX_TRACE
+  unsigned long long* const trace_buf =
+      static_cast<int>(blockIdx.x) == g_trace_cta ? g_trace : nullptr;
+#endif
   // A wait of an earlier CTA already expired: do not start more work.
   if (*reinterpret_cast<volatile unsigned int*>(&g_status) & kStatusTimeout) return;
 
@@ -393,12 +402,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     for (int q = 0; q < 2; ++q) {
       for (int i = 0; i < 2; ++i) {
-        ptx::mbar_init(&bars->s_full[q][i], 1);
         ptx::mbar_init(&bars->p_full[q][i], 128);
         ptx::mbar_init(&bars->pv_done[q][i], 1);
         ptx::mbar_init(&bars->o_ready[q][i], 128);
       }
       ptx::mbar_init(&bars->o_final[q], 1);
+      ptx::mbar_init(&bars->s_full[q], 1);
+      ptx::mbar_init(&bars->s_free[q], 128);
     }
     ptx::mbar_init(&bars->drain[0], 1);
     ptx::mbar_init(&bars->drain[1], 1);
@@ -473,10 +483,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 1 || warp == 2) {
     // ================= MMA issuers: warp 1 for Q tile 0, warp 2 for Q tile 1 =====
-    // Order: S_q(0), S_q(1), then per key tile j: P_q(j).V followed at once by
-    // S_q(j + 2), which reuses the score buffer P_q(j) was read from:
-    // tcgen05.mma operations of one thread run in issue order, so no wait is
-    // needed for that reuse.  A thread whose Q tile is shorter (or absent) still releases
+    // Order: S_q(0), then per key tile j: S_q(j + 1) as soon as the softmax has
+    // read S_q(j) out of TMEM, then P_q(j).V once O_q is ready for it.  A thread whose Q tile is shorter (or absent) still releases
     // the remaining K/V stages, after they are loaded, so that each stage's
     // release barrier sees one arrival per Q tile.
     const int q = warp - 1;
@@ -492,25 +500,43 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint32_t d_o = tmem + S::col_o(q);
       bool ok = wait_bar(&bars->q_full, 0, abort_flag, tmo);
       ptx::tc_fence_after();
-      // S(i) for the first two tiles; afterwards S(j + 2) follows P(j).V at once
-      // so that the score buffer is refilled as early as possible.
-      for (int i = 0; ok && i < 2 && i < ntq; ++i) {
-        const int st = i % kStages;
-        if (!wait_bar(&bars->kv_full[st], (i / kStages) & 1, abort_flag, tmo)) {
-          ok = false;
-          break;
+      const uint32_t d_s = tmem + S::col_s(q);
+      // Every K/V stage of tiles 0 .. nt-1 is awaited exactly once, in order:
+      // before S(i) for tiles this Q tile uses, before the release otherwise.
+#define TILEMIX_KV_WAIT(i) \
+  wait_bar(&bars->kv_full[(i) % kStages], ((i) / kStages) & 1, abort_flag, tmo)
+      if (ntq > 0) {
+        if (!TILEMIX_KV_WAIT(0)) ok = false;
+        if (ok) {
+          ptx::tc_fence_after();
+          issue_qk<D>(d_s, routed_int8(word, 0, gs), aq16, aq8, a_smem + S::kOffK16,
+                      a_smem + S::kOffK8, t16, t8);
+          ptx::mma_commit(&bars->s_full[q]);
+          TRACE(4, q, 0);
         }
-        ptx::tc_fence_after();
-        issue_qk<D>(tmem + S::col_s(q, i & 1), routed_int8(word, i, gs), aq16, aq8,
-                    a_smem + S::kOffK16 + st * S::kK16, a_smem + S::kOffK8 + st * S::kK8, t16,
-                    t8);
-        ptx::mma_commit(&bars->s_full[q][i & 1]);
-        TRACE(4, q, i);
       }
       for (int j = 0; ok && j < nt; ++j) {
         const int st = j % kStages;
+        const int i = j + 1;  // next score tile
+        if (i < ntq) {
+          // S(i) overwrites S(j) once the softmax has read it out
+          if (!wait_bar(&bars->s_free[q], j & 1, abort_flag, tmo) || !TILEMIX_KV_WAIT(i)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const int sti = i % kStages;
+          issue_qk<D>(d_s, routed_int8(word, i, gs), aq16, aq8,
+                      a_smem + S::kOffK16 + sti * S::kK16, a_smem + S::kOffK8 + sti * S::kK8,
+                      t16, t8);
+          ptx::mma_commit(&bars->s_full[q]);
+          TRACE(4, q, i);
+        } else if (i < nt && !TILEMIX_KV_WAIT(i)) {
+          ok = false;
+          break;
+        }
         if (j < ntq) {
-          const int sb = j & 1;
+          const int pb = j & 1;
           const int valid = L - j * BN;
           if (valid < BN) {
             // Keys past the sequence end belong to the next packed sequence:
@@ -525,39 +551,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               }
             ptx::fence_proxy_async_smem();
           }
-          if (!wait_bar(&bars->o_ready[q][sb], (j >> 1) & 1, abort_flag, tmo)) {
+          if (!wait_bar(&bars->o_ready[q][pb], (j >> 1) & 1, abort_flag, tmo)) {
             ok = false;
             break;
           }
           TRACE(10, q, j);
           ptx::tc_fence_after();
-          issue_pv<D>(d_o, tmem + S::col_s(q, sb), a_smem + S::kOffV + st * S::kV, tv, j == 0);
-          TRACE(5, q, j);
-          const int i = j + 2;
-          if (i < ntq) {
-            const int sti = i % kStages;
-            if (!wait_bar(&bars->kv_full[sti], (i / kStages) & 1, abort_flag, tmo)) {
-              ok = false;
-              break;
-            }
-            ptx::tc_fence_after();
-            issue_qk<D>(tmem + S::col_s(q, sb), routed_int8(word, i, gs), aq16, aq8,
-                        a_smem + S::kOffK16 + sti * S::kK16, a_smem + S::kOffK8 + sti * S::kK8,
-                        t16, t8);
-            ptx::mma_commit(&bars->s_full[q][sb]);
-            TRACE(4, q, i);
-          }
-          ptx::mma_commit(&bars->pv_done[q][sb]);
+          issue_pv<D>(d_o, tmem + S::col_p(q, pb), a_smem + S::kOffV + st * S::kV, tv, j == 0);
+          ptx::mma_commit(&bars->pv_done[q][pb]);
           if (j == ntq - 1) ptx::mma_commit(&bars->o_final[q]);
-        } else {
-          // a tile this Q tile does not use: release it once it is loaded
-          if (!wait_bar(&bars->kv_full[st], (j / kStages) & 1, abort_flag, tmo)) {
-            ok = false;
-            break;
-          }
+          TRACE(5, q, j);
         }
         ptx::mma_commit(&bars->kv_empty[st]);
       }
+#undef TILEMIX_KV_WAIT
       // all MMAs of this thread complete before TMEM and shared memory go away
       ptx::mma_commit(&bars->drain[q]);
       drain_bar(&bars->drain[q], 0, tmo);
@@ -584,16 +591,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const bool is_int = routed_int8(t.word, i, gs);
         const float k_sc = k_sc_next;
         if (i + 1 < t.ntiles) k_sc_next = __ldg(ks + i + 1);
-        if (!wait_bar_warp(&bars->s_full[q][sb], (i >> 1) & 1, abort_flag, tmo)) {
+        if (!wait_bar_warp(&bars->s_full[q], i & 1, abort_flag, tmo)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         if (tr == 0) TRACE(0, q, i);
-        const uint32_t ts = tmem + lane_base + S::col_s(q, sb);
+        const uint32_t ts = tmem + lane_base + S::col_s(q);
         ptx::tmem_ld32(ts, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         ptx::tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         ptx::tmem_ld_wait();
+        // S(i) is in registers: the MMA warp may compute S(i + 1) now
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->s_free[q]);
         if (tr == 0) TRACE(11, q, i);
         if (is_int && p.dbg && my_row < L) {
           int32_t* drow =
@@ -659,7 +669,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (tr == 0) TRACE(15, q, i);
         // the correction warps rescale O by alpha before P(i).V is issued
         alpha_smem[(q * 2 + sb) * BM + tr] = (i > 0) ? alpha : 1.0f;
-        ptx::tmem_st32(ts, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
+        // P buffer sb held P(i - 2): wait until P(i - 2).V has read it
+        if (i >= 2 &&
+            !wait_bar_warp(&bars->pv_done[q][sb], ((i - 2) >> 1) & 1, abort_flag, tmo)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        ptx::tmem_st32(tmem + lane_base + S::col_p(q, sb),
+                       *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[q][sb]);
