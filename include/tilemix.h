@@ -55,7 +55,8 @@ typedef enum {
   TILEMIX_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. head dim not 64/128) */
   TILEMIX_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
   TILEMIX_ERR_TIMEOUT = 4,      /* a bounded device wait expired; outputs undefined */
-  TILEMIX_ERR_WORKSPACE = 5     /* workspace missing or smaller than required */
+  TILEMIX_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required */
+  TILEMIX_ERR_TOO_LARGE = 6     /* needs more scratch than tilemix_prefill_fwd_noalloc has */
 } tilemix_status;
 
 typedef enum {
@@ -178,6 +179,31 @@ int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes);
  * Enqueues the K quantisation pre-pass (unless k_i8 is given), the Q
  * quantisation and the fused attention kernel on `stream`. */
 int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
+
+/* Allocation-free variant of tilemix_prefill_fwd.  (The TileMix pages have no
+ * counterpart: this is a deployment convenience of this library.)
+ *
+ * For callers that cannot call cudaMalloc or any allocator at this point: for
+ * example code running inside a host application that owns all device memory
+ * through its own pool and forbids side allocations, or a latency-critical
+ * path where an allocation, which may synchronise the device, is not allowed.
+ * The caller still passes q, k, v, o (and the other tensors) as for
+ * tilemix_prefill_fwd; args->workspace and args->workspace_bytes are ignored.
+ * The INT8 codes and scales that tilemix_prefill_fwd keeps in the caller's
+ * workspace live instead in one fixed scratch array of 64 MiB inside the
+ * library (TILEMIX_NOALLOC_SCRATCH_BYTES), which every GPU that loads the
+ * library holds until the process exits.  A call whose workspace would exceed
+ * it (tilemix_workspace_size() > 64 MiB) returns TILEMIX_ERR_TOO_LARGE and
+ * launches nothing.  Results equal those of tilemix_prefill_fwd.
+ *
+ * The first call on a device looks up the scratch array's device address
+ * (once per device, with that device current); make that first call before
+ * any stream capture.  All calls share the one array: calls that overlap on
+ * the GPU (on different streams, or from different threads) race on it and
+ * must be serialised by the caller.  Nothing in the array needs to start at
+ * zero; every call rewrites what it reads. */
+#define TILEMIX_NOALLOC_SCRATCH_BYTES (64u << 20)
+int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word:
  * OK, TIMEOUT (a bounded wait expired), INVALID_ARG (a row needed more than 64

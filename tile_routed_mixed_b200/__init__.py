@@ -21,7 +21,8 @@ BLOCK_M = 128
 BLOCK_N = 64
 MAX_GROUPS = 64
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_TOO_LARGE = range(7)
+NOALLOC_SCRATCH_BYTES = 64 << 20
 TEMPLATES = {"band": 0, "global": 1, "row_random": 2, "aligned_sparse": 3, "bigbird": 4,
              "sptrans": 5}
 
@@ -79,6 +80,8 @@ def lib():
                                              ctypes.POINTER(ctypes.c_size_t)]
         L.tilemix_prefill_fwd.restype = I
         L.tilemix_prefill_fwd.argtypes = [ctypes.POINTER(PrefillArgs), P]
+        L.tilemix_prefill_fwd_noalloc.restype = I
+        L.tilemix_prefill_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), P]
         L.tilemix_get_error.restype = I
         L.tilemix_get_error.argtypes = [P]
         _lib = L
@@ -211,6 +214,13 @@ def tilemix_prefill_fwd(args: PrefillArgs, stream=None):
            "tilemix_prefill_fwd")
 
 
+def tilemix_prefill_fwd_noalloc(args: PrefillArgs, stream=None):
+    """tilemix_prefill_fwd without a caller workspace: the library's fixed
+    64 MiB scratch array is used instead (see include/tilemix.h)."""
+    _check(lib().tilemix_prefill_fwd_noalloc(ctypes.byref(args), _stream_handle(stream)),
+           "tilemix_prefill_fwd_noalloc")
+
+
 def tilemix_get_error(stream=None) -> int:
     return int(lib().tilemix_get_error(_stream_handle(stream)))
 
@@ -220,7 +230,8 @@ from .prefill import TileMixPrefill  # noqa: E402  (convenience wrapper)
 __all__ = [
     "BLOCK_M", "BLOCK_N", "MAX_GROUPS", "PrefillArgs", "TEMPLATES", "TileMixError",
     "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
-    "tilemix_build_routing", "tilemix_get_error", "tilemix_prefill_fwd", "tilemix_quantize_qk",
+    "tilemix_build_routing", "tilemix_get_error", "tilemix_prefill_fwd",
+    "tilemix_prefill_fwd_noalloc", "tilemix_quantize_qk",
     "tilemix_status_string", "tilemix_tile_offsets", "tilemix_version",
     "tilemix_workspace_size",
 ]

@@ -122,6 +122,8 @@ TILEMIX_API const char* tilemix_status_string(int status) {
     case TILEMIX_ERR_CUDA: return "CUDA error";
     case TILEMIX_ERR_TIMEOUT: return "device wait timed out";
     case TILEMIX_ERR_WORKSPACE: return "workspace missing or too small";
+    case TILEMIX_ERR_TOO_LARGE:
+      return "workspace needed exceeds the 64 MiB scratch of tilemix_prefill_fwd_noalloc";
     default: return "unknown status";
   }
 }
@@ -239,6 +241,19 @@ TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream)
       cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_end), st) != cudaSuccess)
     return TILEMIX_ERR_CUDA;
   return TILEMIX_OK;
+}
+
+TILEMIX_API int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream) {
+  int rc = check_args(args);
+  if (rc != TILEMIX_OK) return rc;
+  if (args->nseq == 0 || args->total_tokens == 0) return TILEMIX_OK;
+  if (layout_of(args).total > TILEMIX_NOALLOC_SCRATCH_BYTES) return TILEMIX_ERR_TOO_LARGE;
+  void* scratch = nullptr;
+  if (tilemix::noalloc_scratch(&scratch) != cudaSuccess) return TILEMIX_ERR_CUDA;
+  tilemix_prefill_args a = *args;
+  a.workspace = scratch;
+  a.workspace_bytes = TILEMIX_NOALLOC_SCRATCH_BYTES;
+  return tilemix_prefill_fwd(&a, stream);
 }
 
 TILEMIX_API int tilemix_get_error(void* stream) {

@@ -48,5 +48,8 @@ int launch_quantize(const void* x, const int32_t* cu_seqlens, const int32_t* cu_
                     float* scales, cudaStream_t stream);
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
 int read_and_clear_status(unsigned int* status, cudaStream_t stream);
+// Device address of the allocation-free entry point's scratch array on the
+// current device (looked up once per device).
+int noalloc_scratch(void** ptr);
 
 }  // namespace tilemix

@@ -14,6 +14,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
+#include "tilemix.h"
 #include "tilemix_internal.h"
 #include "tilemix_ptx.cuh"
 
@@ -781,6 +784,31 @@ extern "C" TILEMIX_API int tilemix_trace_setup(void* buf, int cta) {
   return cudaMemcpyToSymbol(g_trace_cta, &cta, sizeof(cta)) != cudaSuccess;
 }
 #endif
+
+// Scratch of the allocation-free entry point: module-scope device memory,
+// present on every GPU that loads this library.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TILEMIX_NOALLOC_SCRATCH_BYTES];
+
+int noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  // Device address of the array, looked up once per device (host code cannot
+  // take the symbol's address directly).
+  static std::mutex mu;
+  static void* cached[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cached[dev]) {
+    *ptr = cached[dev];
+    return cudaSuccess;
+  }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  if (dev >= 0 && dev < 64) cached[dev] = p;
+  *ptr = p;
+  return cudaSuccess;
+}
 
 int read_and_clear_status(unsigned int* status, cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
