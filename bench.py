@@ -159,6 +159,41 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity when not
+    distributed).  Timing of multi-GPU runs is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_tokens(tokens_per_rank, world):
+    """Weak scaling: every rank processes its own full batch."""
+    return int(tokens_per_rank) * int(world)
+
+
+def kernel_traffic(workload_name):
+    """DRAM bytes per launch of the fused kernel from the committed ncu record,
+    or None if the record is for another workload or the kernel source changed
+    since it was captured."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)["prefill_fwd_kernel<128>"]
+        h = hashlib.sha256()
+        for name in ("tilemix_kernels.cu", "tilemix_ptx.cuh"):
+            with open(os.path.join(ROOT, "tile_routed_mixed_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        if rec["workload"] != workload_name or h.hexdigest()[:16] != rec["kernel_source_sha256_16"]:
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def host_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -199,7 +234,7 @@ def cpu_baseline(q, k, v, lengths, hq, hk, masks, g, causal, budget_s=15.0):
     T = sum(lengths)
     cal = random_rows(lengths, hq, 256, rng)
     t_cal, t_quant, quant = oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, cal)
-    n = int(max(256, min(200000, 256 * budget_s / max(t_cal, 1e-3))))
+    n = int(max(256, min(1000000, 256 * budget_s / max(t_cal, 1e-3))))
     rows = random_rows(lengths, hq, n, rng)
     t_rows, _, _ = oracle_sample(q, k, v, lengths, hq, hk, masks, g, causal, rows, quant=quant)
     t = t_rows + t_quant * n / (T * hq)
@@ -324,10 +359,7 @@ def run_gpu(args):
         raise tm.TileMixError(rc, "timed steps")
     ms = e0.elapsed_time(e1) / args.steps
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    t = torch.tensor([ms, kern_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, kern_ms = float(t[0]), float(t[1])
+    ms, kern_ms = max_over_ranks([ms, kern_ms], device=dev)
 
     # end to end through the public call with pinned host buffers
     qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
@@ -350,13 +382,10 @@ def run_gpu(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], device=dev)[0]
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.barrier()
         dist.destroy_process_group()
-    e2e_ms = float(t[0])
     if rank != 0:
         return
 
@@ -373,7 +402,7 @@ def run_gpu(args):
         peak, unit = p16 / 1e12, "TFLOP/s"
     else:
         achieved, peak, unit = nbytes / t_k / 1e9, pk["hbm_gbs"], "GB/s"
-    tokens = T * world
+    tokens = whole_job_tokens(T, world)
     line = {
         "metric": METRIC,
         "value": tokens / (ms / 1e3),
@@ -390,7 +419,8 @@ def run_gpu(args):
         "config": bench_config(args, w, lengths, g),
         "roofline": {
             "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": None,
+            "frac": achieved / peak, "traffic": kernel_traffic(args.workload),
+            "traffic_unit": "bytes per launch (ncu)",
             "kernel": "prefill_fwd_kernel<128>",
             "kernel_ms": kern_ms,
             "peak_kind": "burst (%s)" % pk["source"],
@@ -413,7 +443,7 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=1500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["tilemix", "reference"], default="tilemix")
     ap.add_argument("--workload", default="llama3b_4k_b8", choices=list(synth.WORKLOADS))

@@ -205,6 +205,13 @@ int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
 #define TILEMIX_NOALLOC_SCRATCH_BYTES (64u << 20)
 int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
 
+/* Self test of the failure path: enqueues one warp that waits on a device
+ * barrier nothing ever signals, with the same bounded wait the attention
+ * kernel uses, limited to timeout_ms (1..10000).  The wait gives up, latches
+ * TILEMIX_ERR_TIMEOUT in the device status word and the kernel returns; the
+ * CUDA context stays usable.  INVALID_ARG for an out-of-range timeout. */
+int tilemix_selftest_wait_timeout(int timeout_ms, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word:
  * OK, TIMEOUT (a bounded wait expired), INVALID_ARG (a row needed more than 64
  * groups, or a bad routing-group factor), or CUDA for a sticky CUDA error. */

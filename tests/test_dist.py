@@ -1,0 +1,46 @@
+"""Multi-rank plumbing of bench.py on CPU (gloo, world size 2): ranks time
+their own batch (weak scaling, no collective on the data path) and the job's
+time is the slowest rank's."""
+import os
+import socket
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import bench
+    ms, kern = bench.max_over_ranks([1.0 + rank, 5.0 - rank])
+    out[rank] = (ms, kern, bench.whole_job_tokens(32768, world))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world_2(root):
+    world = 2
+    port = _free_port()
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True,
+                       start_method="spawn")
+    assert dict(out) == {0: (2.0, 5.0, 65536), 1: (2.0, 5.0, 65536)}
+
+
+def test_single_process_is_identity():
+    import bench
+    assert bench.max_over_ranks([3.5, 1.25]) == [3.5, 1.25]
+    assert bench.whole_job_tokens(32768, 1) == 32768

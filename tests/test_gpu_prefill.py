@@ -213,3 +213,37 @@ def test_workload_sampled_rows(name, over):
         rows = gc.sample_rows(case.lengths, case.hq, per_head_random=32)
     want, _, _ = gc.oracle_rows(case, q, k, v, masks, rows)
     _check_out(case, out["o"], want, rows)
+
+
+# ------------------------------------------------------------- failures ---
+
+def test_bounded_wait_expires_and_is_reported():
+    # a barrier nothing signals: the wait gives up after 50 ms, the status
+    # word reports TIMEOUT once, and the context still runs the kernel
+    import tile_routed_mixed_b200 as tm
+    tm.tilemix_selftest_wait_timeout(50)
+    assert tm.tilemix_get_error() == tm.ERR_TIMEOUT
+    assert tm.tilemix_get_error() == tm.OK
+    case = gc.Case([200], 2, 1, 64, template="band", percent=50)
+    q, k, v = case.inputs()
+    masks = case.masks()
+    out = gc.run_gpu(case, q, k, v, masks)
+    rows = oracle.all_rows(case.lengths, case.hq)
+    want, _, _ = gc.oracle_rows(case, q, k, v, masks, rows)
+    _check_out(case, out["o"], want, rows)
+    with pytest.raises(tm.TileMixError):
+        tm.tilemix_selftest_wait_timeout(0)
+
+
+def test_row_with_too_many_groups_is_reported():
+    # g = 1 on an 8192-token sequence needs 128 groups per row: the device
+    # rejects the rows it cannot encode and reports INVALID_ARG
+    import tile_routed_mixed_b200 as tm
+    case = gc.Case([8192], 1, 1, 64, template="band", percent=0, g=2)
+    q, k, v = case.inputs()
+    masks = case.masks()
+    bad = gc.Case([8192], 1, 1, 64, template="band", percent=0, g=1)
+    with pytest.raises(tm.TileMixError) as e:
+        gc.run_gpu(bad, q, k, v, masks)
+    assert e.value.status == tm.ERR_INVALID_ARG
+    assert tm.tilemix_get_error() == tm.OK

@@ -82,6 +82,8 @@ def lib():
         L.tilemix_prefill_fwd.argtypes = [ctypes.POINTER(PrefillArgs), P]
         L.tilemix_prefill_fwd_noalloc.restype = I
         L.tilemix_prefill_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), P]
+        L.tilemix_selftest_wait_timeout.restype = I
+        L.tilemix_selftest_wait_timeout.argtypes = [I, P]
         L.tilemix_get_error.restype = I
         L.tilemix_get_error.argtypes = [P]
         _lib = L
@@ -221,6 +223,11 @@ def tilemix_prefill_fwd_noalloc(args: PrefillArgs, stream=None):
            "tilemix_prefill_fwd_noalloc")
 
 
+def tilemix_selftest_wait_timeout(timeout_ms: int, stream=None):
+    _check(lib().tilemix_selftest_wait_timeout(int(timeout_ms), _stream_handle(stream)),
+           "tilemix_selftest_wait_timeout")
+
+
 def tilemix_get_error(stream=None) -> int:
     return int(lib().tilemix_get_error(_stream_handle(stream)))
 
@@ -231,7 +238,7 @@ __all__ = [
     "BLOCK_M", "BLOCK_N", "MAX_GROUPS", "PrefillArgs", "TEMPLATES", "TileMixError",
     "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
     "tilemix_build_routing", "tilemix_get_error", "tilemix_prefill_fwd",
-    "tilemix_prefill_fwd_noalloc", "tilemix_quantize_qk",
+    "tilemix_prefill_fwd_noalloc", "tilemix_quantize_qk", "tilemix_selftest_wait_timeout",
     "tilemix_status_string", "tilemix_tile_offsets", "tilemix_version",
     "tilemix_workspace_size",
 ]

@@ -256,6 +256,14 @@ TILEMIX_API int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, vo
   return tilemix_prefill_fwd(&a, stream);
 }
 
+TILEMIX_API int tilemix_selftest_wait_timeout(int timeout_ms, void* stream) {
+  if (timeout_ms < 1 || timeout_ms > 10000) return TILEMIX_ERR_INVALID_ARG;
+  if (tilemix::launch_selftest_wait(static_cast<unsigned long long>(timeout_ms) * 1000000ull,
+                                    static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  return TILEMIX_OK;
+}
+
 TILEMIX_API int tilemix_get_error(void* stream) {
   unsigned int status = 0;
   if (tilemix::read_and_clear_status(&status, static_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -51,5 +51,6 @@ int read_and_clear_status(unsigned int* status, cudaStream_t stream);
 // Device address of the allocation-free entry point's scratch array on the
 // current device (looked up once per device).
 int noalloc_scratch(void** ptr);
+int launch_selftest_wait(unsigned long long timeout_ns, cudaStream_t stream);
 
 }  // namespace tilemix

@@ -785,6 +785,25 @@ extern "C" TILEMIX_API int tilemix_trace_setup(void* buf, int cta) {
 }
 #endif
 
+// Failure-path self test: one warp waits on an mbarrier that nothing ever
+// arrives on; the bounded wait must give up and latch kStatusTimeout.
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  wait_bar(&bar, 0, &abort_flag, timeout_ns);
+}
+
+int launch_selftest_wait(unsigned long long timeout_ns, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(timeout_ns);
+  return static_cast<int>(cudaGetLastError());
+}
+
 // Scratch of the allocation-free entry point: module-scope device memory,
 // present on every GPU that loads this library.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[TILEMIX_NOALLOC_SCRATCH_BYTES];
