@@ -203,8 +203,9 @@ struct Smem {
 // unambiguous when the waiter is at most one phase behind the barrier, so each
 // barrier is sized so that this holds.  S is single-buffered: S(i+1) needs
 // s_free(i), which needs the softmax to have read S(i).  P is double-buffered
-// and the softmax stores P(i) only after P(i-2).V completed, so the
-// correction cannot fall two phases behind p_full, and every waiter of
+// and the softmax stores P(i) only after S(i) landed, whose commit follows
+// P(i-2).V (issued earlier by the same thread), so P(i-2).V has completed:
+// the correction cannot fall two phases behind p_full, and every waiter of
 // pv_done / o_ready is at most one phase behind.
 struct Barriers {
   uint64_t q_full;
@@ -270,9 +271,18 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-__device__ __forceinline__ bool routed_int8(uint64_t word, int kt, int g) {
-  return (word >> (kt / g)) & 1ull;
-}
+// Routing lookup along consecutive key tiles: group = tile / g, tracked
+// incrementally (no division in the hot loops); the bit is a shift and a mask.
+struct GroupCursor {
+  int group = 0, in_group = 0;
+  __device__ __forceinline__ bool int8(uint64_t word) const { return (word >> group) & 1ull; }
+  __device__ __forceinline__ void next(int g) {
+    if (++in_group == g) {
+      in_group = 0;
+      ++group;
+    }
+  }
+};
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float m;
@@ -333,14 +343,6 @@ __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint32_t vb
                     (!first || kk > 0) ? 1u : 0u);
 }
 
-// Per-Q-tile geometry of a CTA.
-struct QTile {
-  int qt;        // query-tile row inside the sequence
-  int row0;      // first query row
-  int ntiles;    // legal key tiles (0 if this Q tile does not exist)
-  uint64_t word; // routing word of (row, KV head)
-};
-
 template <int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ PrefillParams p) {
@@ -370,29 +372,24 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (2 * pair >= tm) return;
   const int kv = p.kv_head_of_q ? p.kv_head_of_q[h] : h / p.group;
   const int gs = p.g[s];
-  QTile qtile[2];
-  int nt = 0;
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    QTile& t = qtile[q];
-    t.qt = 2 * pair + q;
-    t.row0 = t.qt * BM;
-    if (t.qt < tm) {
-      // causal and boundary legality: independent of the routing word
-      const int last = p.causal ? (min(t.row0 + BM, L) - 1) / BN : (L - 1) / BN;
-      t.ntiles = last + 1;
-      t.word = p.masks[static_cast<size_t>(p.cu_qtiles[s] + t.qt) * p.hk + kv];
-    } else {
-      t.ntiles = 0;
-      t.word = 0;
-    }
-    nt = max(nt, t.ntiles);
-  }
+  // The CTA's two Q tiles: query-tile rows 2 pair and 2 pair + 1 (the second
+  // may not exist).  Causal and boundary legality fix each row's key-tile
+  // count, independently of the routing words.
+  const int qt0 = 2 * pair;
+  const int last0 = p.causal ? (min(qt0 * BM + BM, L) - 1) / BN : (L - 1) / BN;
+  const int nt0 = last0 + 1;
+  const bool has1 = qt0 + 1 < tm;
+  const int last1 = p.causal ? (min(qt0 * BM + 2 * BM, L) - 1) / BN : (L - 1) / BN;
+  const int nt1 = has1 ? last1 + 1 : 0;
+  const uint64_t* wrow = p.masks + static_cast<size_t>(p.cu_qtiles[s] + qt0) * p.hk + kv;
+  const uint64_t w0 = wrow[0];
+  const uint64_t w1 = has1 ? wrow[p.hk] : 0ull;
+  const int nt = max(nt0, nt1);
   if (gs < 1 || (nt - 1) / gs > 63) {
     if (threadIdx.x == 0) atomicOr(&g_status, kStatusBadGroups);
     return;
   }
-  const int nq = qtile[1].ntiles > 0 ? 2 : 1;
+  const int nq = has1 ? 2 : 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -442,24 +439,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       ptx::prefetch_tensormap(&p.tm_v);
       ptx::mbar_expect_tx(&bars->q_full, nq * (S::kQ + S::kQ8));
       for (int q = 0; q < nq; ++q) {
+        const int row = t0 + (qt0 + q) * BM;
 #pragma unroll
         for (int j = 0; j < D / 64; ++j)
           ptx::tma_load_3d(smem + S::kOffQ + q * S::kQ + j * BM * 128, &p.tm_q, &bars->q_full,
-                           j * 64, h, t0 + qtile[q].row0);
-        ptx::tma_load_3d(smem + S::kOffQ8 + q * S::kQ8, &p.tm_q8, &bars->q_full, 0, h,
-                         t0 + qtile[q].row0);
+                           j * 64, h, row);
+        ptx::tma_load_3d(smem + S::kOffQ8 + q * S::kQ8, &p.tm_q8, &bars->q_full, 0, h, row);
       }
-      int cnt[kStages] = {};
-      for (int i = 0; i < nt; ++i) {
+      int issued = 0;
+      GroupCursor gc;
+      for (int i = 0; i < nt; ++i, gc.next(gs)) {
         const int st = i % kStages;
-        bool need16 = false, need8 = false;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          if (i < qtile[q].ntiles) {
-            if (routed_int8(qtile[q].word, i, gs)) need8 = true;
-            else need16 = true;
-          }
-        }
+        // K precisions the two rows need for this tile
+        const bool b0 = gc.int8(w0), b1 = gc.int8(w1);
+        const bool need8 = (i < nt0 && b0) || (i < nt1 && b1);
+        const bool need16 = (i < nt0 && !b0) || (i < nt1 && !b1);
         if (i >= kStages && !wait_bar(&bars->kv_empty[st], ((i / kStages) - 1) & 1, abort_flag, tmo))
           break;
         const int key0 = t0 + i * BN;
@@ -477,12 +471,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int j = 0; j < D / 64; ++j)
           ptx::tma_load_3d(smem + S::kOffV + st * S::kV + j * BN * 128, &p.tm_v, full, j * 64, kv,
                            key0);
-        ++cnt[st];
+        ++issued;
       }
       // Never leave with copies into this CTA's shared memory in flight.
       drain_bar(&bars->q_full, 0, tmo);
-      for (int st = 0; st < kStages; ++st)
-        if (cnt[st]) drain_bar(&bars->kv_full[st], (cnt[st] - 1) & 1, tmo);
+      for (int st = 0; st < kStages && st < issued; ++st)
+        drain_bar(&bars->kv_full[st], ((issued - 1 - st) / kStages) & 1, tmo);
     }
   } else if (warp == 1 || warp == 2) {
     // ================= MMA issuers: warp 1 for Q tile 0, warp 2 for Q tile 1 =====
@@ -496,8 +490,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint64_t t16 = ptx::smem_desc(0, 16, 1024, ptx::kSwizzle128B);
       const uint64_t t8 = ptx::smem_desc(0, 16, S::kI8Sbo, S::kI8Layout);
       const uint64_t tv = ptx::smem_desc(0, BN * 128, 1024, ptx::kSwizzle128B);
-      const int ntq = qtile[q].ntiles;
-      const uint64_t word = qtile[q].word;
+      const int ntq = q ? nt1 : nt0;
+      const uint64_t word = q ? w1 : w0;
       const uint32_t aq16 = a_smem + S::kOffQ + q * S::kQ;
       const uint32_t aq8 = a_smem + S::kOffQ8 + q * S::kQ8;
       const uint32_t d_o = tmem + S::col_o(q);
@@ -508,15 +502,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // before S(i) for tiles this Q tile uses, before the release otherwise.
 #define TILEMIX_KV_WAIT(i) \
   wait_bar(&bars->kv_full[(i) % kStages], ((i) / kStages) & 1, abort_flag, tmo)
+      GroupCursor gc;  // routing group of the next score tile
       if (ntq > 0) {
         if (!TILEMIX_KV_WAIT(0)) ok = false;
         if (ok) {
           ptx::tc_fence_after();
-          issue_qk<D>(d_s, routed_int8(word, 0, gs), aq16, aq8, a_smem + S::kOffK16,
-                      a_smem + S::kOffK8, t16, t8);
+          issue_qk<D>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16, a_smem + S::kOffK8,
+                      t16, t8);
           ptx::mma_commit(&bars->s_full[q]);
           TRACE(4, q, 0);
         }
+        gc.next(gs);
       }
       for (int j = 0; ok && j < nt; ++j) {
         const int st = j % kStages;
@@ -529,10 +525,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           ptx::tc_fence_after();
           const int sti = i % kStages;
-          issue_qk<D>(d_s, routed_int8(word, i, gs), aq16, aq8,
-                      a_smem + S::kOffK16 + sti * S::kK16, a_smem + S::kOffK8 + sti * S::kK8,
-                      t16, t8);
+          issue_qk<D>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16 + sti * S::kK16,
+                      a_smem + S::kOffK8 + sti * S::kK8, t16, t8);
           ptx::mma_commit(&bars->s_full[q]);
+          gc.next(gs);
           TRACE(4, q, i);
         } else if (i < nt && !TILEMIX_KV_WAIT(i)) {
           ok = false;
@@ -578,22 +574,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int q = (warp - kSoftmaxWarp0) >> 2;        // Q tile of this warpgroup
     const int tr = threadIdx.x - (kSoftmaxWarp0 + 4 * q) * 32;  // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const QTile t = qtile[q];
-    const int my_row = t.row0 + tr;
-    if (t.ntiles > 0) {
+    const int ntq = q ? nt1 : nt0;
+    const uint64_t word = q ? w1 : w0;
+    const int row0 = (qt0 + q) * BM;
+    const int my_row = row0 + tr;
+    if (ntq > 0) {
       const float q_sc =
-          p.q_scale[static_cast<size_t>(h) * p.total_qtiles + p.cu_qtiles[s] + t.qt];
+          p.q_scale[static_cast<size_t>(h) * p.total_qtiles + p.cu_qtiles[s] + qt0 + q];
       const float* ks = p.k_scale + static_cast<size_t>(kv) * p.total_ktiles + p.cu_ktiles[s];
       float m = -INFINITY;  // running max, log2 units
       float l = 0.f;        // normaliser: sum of the fp16-rounded P actually used in P.V
       bool ok = true;
       uint32_t r[64];
       float k_sc_next = __ldg(ks);
-      for (int i = 0; i < t.ntiles; ++i) {
+      GroupCursor gc;
+      for (int i = 0; i < ntq; ++i, gc.next(gs)) {
         const int sb = i & 1;
-        const bool is_int = routed_int8(t.word, i, gs);
+        const bool is_int = gc.int8(word);
         const float k_sc = k_sc_next;
-        if (i + 1 < t.ntiles) k_sc_next = __ldg(ks + i + 1);
+        if (i + 1 < ntq) k_sc_next = __ldg(ks + i + 1);
         if (!wait_bar_warp(&bars->s_full[q], i & 1, abort_flag, tmo)) {
           ok = false;
           break;
@@ -622,7 +621,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         const float c = is_int ? q_sc * k_sc * p.scale_log2 : p.scale_log2;
         const int key0 = i * BN;
-        const bool masked = key0 + BN > L || (p.causal && key0 + BN - 1 > t.row0);
+        const bool masked = key0 + BN > L || (p.causal && key0 + BN - 1 > row0);
         const int lim = p.causal ? min(L, my_row + 1) : L;  // legal keys < lim
         if (masked) {
 #pragma unroll
@@ -672,13 +671,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (tr == 0) TRACE(15, q, i);
         // the correction warps rescale O by alpha before P(i).V is issued
         alpha_smem[(q * 2 + sb) * BM + tr] = (i > 0) ? alpha : 1.0f;
-        // P buffer sb held P(i - 2): wait until P(i - 2).V has read it
-        if (i >= 2 &&
-            !wait_bar_warp(&bars->pv_done[q][sb], ((i - 2) >> 1) & 1, abort_flag, tmo)) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
+        // P buffer sb held P(i - 2).  Its P.V was issued before S(i) by the
+        // same thread, and the commit that signalled S(i) covers every MMA
+        // issued before it, so P(i - 2).V has completed: no wait needed.
         ptx::tmem_st32(tmem + lane_base + S::col_p(q, sb),
                        *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
         ptx::tmem_st_wait();
@@ -719,7 +714,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int q = (warp - kCorrectionWarp0) >> 2;  // Q tile of this warpgroup
     const int tr = threadIdx.x - (kCorrectionWarp0 + 4 * q) * 32;  // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int ntq = qtile[q].ntiles;
+    const int ntq = q ? nt1 : nt0;
     uint32_t r[32];
     for (int i = 0; i < ntq; ++i) {
       const int sb = i & 1;
