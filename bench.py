@@ -432,7 +432,7 @@ def run_gpu(args):
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": int(q.nbytes + k.nbytes + v.nbytes),
                 "d2h_bytes_per_step": int(q.nbytes)},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,  # quantiser + fused attention
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -58,6 +58,60 @@ def test_quantize_bit_exact(lengths, hq, hk, d):
     assert np.array_equal(ks.cpu().numpy().view(np.uint32), kso.view(np.uint32))
 
 
+def _near_half_integers(lengths, heads, d, block, seed):
+    """fp16 values whose quotient x / s sits on or next to a half-integer, per
+    block: the rounding cases where a reciprocal-multiply shortcut and the
+    IEEE quotient can disagree.  One block in three has a = 127 (s = 1, so the
+    ties are exact and rne must pick the even code)."""
+    rng = np.random.default_rng(seed)
+    T = sum(lengths)
+    x = np.zeros((T, heads, d), dtype=np.float16)
+    t0 = 0
+    for L in lengths:
+        for r0 in range(0, L, block):
+            rows = min(block, L - r0)
+            for h in range(heads):
+                a = np.float16(127.0) if rng.integers(3) == 0 else np.float16(rng.uniform(0.05, 9.0))
+                s = np.float32(np.float32(a) / np.float32(127.0))
+                kk = rng.integers(-127, 127, size=(rows, d))
+                tgt = ((kk + 0.5) * np.float64(s)).astype(np.float16)
+                bump = rng.integers(-1, 2, size=(rows, d))
+                up = np.nextafter(tgt, np.float16(np.inf))
+                dn = np.nextafter(tgt, np.float16(-np.inf))
+                v = np.where(bump > 0, up, np.where(bump < 0, dn, tgt))
+                v = np.clip(v, -a, a)
+                v[0, 0] = a
+                x[t0 + r0:t0 + r0 + rows, h, :] = v
+        t0 += L
+    return x
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_quantize_rounding_boundaries_bit_exact(d):
+    import tile_routed_mixed_b200 as tm
+    lengths, hq, hk = [256, 77, 130], 3, 2
+    q = _near_half_integers(lengths, hq, d, 128, seed=11)
+    k = _near_half_integers(lengths, hk, d, 64, seed=12)
+    q8o, qso = oracle.quantize_q(q, lengths)
+    k8o, kso = oracle.quantize_k(k, lengths)
+    cu = synth.cu_seqlens_of(lengths)
+    cq, ck = tm.tilemix_tile_offsets(cu)
+    dev = "cuda"
+    T = sum(lengths)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    q8 = torch.zeros((T, hq, d), dtype=torch.int8, device=dev)
+    k8 = torch.zeros((T, hk, d), dtype=torch.int8, device=dev)
+    qs = torch.zeros((hq, int(cq[-1])), dtype=torch.float32, device=dev)
+    ks = torch.zeros((hk, int(ck[-1])), dtype=torch.float32, device=dev)
+    tm.tilemix_quantize_qk(t(q), t(k), t(cu), t(cq), t(ck), len(lengths), T, int(cq[-1]),
+                           int(ck[-1]), hq, hk, d, q8, qs, k8, ks)
+    torch.cuda.synchronize()
+    assert np.array_equal(q8.cpu().numpy(), q8o)
+    assert np.array_equal(k8.cpu().numpy(), k8o)
+    assert np.array_equal(qs.cpu().numpy().view(np.uint32), qso.view(np.uint32))
+    assert np.array_equal(ks.cpu().numpy().view(np.uint32), kso.view(np.uint32))
+
+
 # --------------------------------------------------------- INT32 scores ---
 
 @pytest.mark.parametrize("case", [

@@ -144,18 +144,16 @@ TILEMIX_API int tilemix_quantize_qk(const void* q_f16, const void* k_f16,
     if (hq < 1 || !cu_qtiles_d || !q_i8 || !q_scale || !aligned16(q_f16) ||
         (reinterpret_cast<uintptr_t>(q_i8) & 7u))
       return TILEMIX_ERR_INVALID_ARG;
-    if (tilemix::launch_quantize(q_f16, cu_seqlens_d, cu_qtiles_d, nseq, total_qtiles, hq, d,
-                                 TILEMIX_BLOCK_M, q_i8, q_scale, st) != cudaSuccess)
-      return TILEMIX_ERR_CUDA;
   }
   if (k_f16) {
     if (hk < 1 || !cu_ktiles_d || !k_i8 || !k_scale || !aligned16(k_f16) ||
         (reinterpret_cast<uintptr_t>(k_i8) & 7u))
       return TILEMIX_ERR_INVALID_ARG;
-    if (tilemix::launch_quantize(k_f16, cu_seqlens_d, cu_ktiles_d, nseq, total_ktiles, hk, d,
-                                 TILEMIX_BLOCK_N, k_i8, k_scale, st) != cudaSuccess)
-      return TILEMIX_ERR_CUDA;
   }
+  if (tilemix::launch_quantize_qk(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq,
+                                  total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8,
+                                  k_scale, st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
   return TILEMIX_OK;
 }
 

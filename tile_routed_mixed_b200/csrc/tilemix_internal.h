@@ -43,9 +43,12 @@ struct PrefillParams {
 };
 
 // Launchers implemented in the CUDA translation unit.  Return cudaError_t.
-int launch_quantize(const void* x, const int32_t* cu_seqlens, const int32_t* cu_tiles, int nseq,
-                    int total_tiles, int heads, int d, int block_rows, int8_t* codes,
-                    float* scales, cudaStream_t stream);
+// One launch quantises Q (128-row blocks) and K (64-row blocks); a null q or
+// k skips that side.
+int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
+                       const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
+                       int total_qtiles, int total_ktiles, int hq, int hk, int d, int8_t* q8,
+                       float* q_scale, int8_t* k8, float* k_scale, cudaStream_t stream);
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
 int read_and_clear_status(unsigned int* status, cudaStream_t stream);
 // Device address of the allocation-free entry point's scratch array on the

@@ -1,6 +1,6 @@
 // CUDA kernels of the tile-routed FP16/INT8 causal prefill attention (sm_100a).
 //
-//   quantize_blocks_kernel   per-(head, block) symmetric absmax/127 INT8 codes
+//   quantize_qk_kernel       per-(head, block) symmetric absmax/127 INT8 codes
 //   prefill_fwd_kernel       fused attention: TMA -> tcgen05 kind::f16 or
 //                            kind::i8 QK^T per key tile (chosen by the routing
 //                            bit) -> shared online softmax -> kind::f16 P.V
@@ -45,89 +45,133 @@ constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 64;   // keys per tile
 
 // ===================================================================
-// Block quantisation.  One CTA per (block, head): pass 1 finds the absmax of
-// the block's valid rows, pass 2 writes codes = clamp(rne(x / s), +-127) with
-// s = a / 127 in IEEE fp32 ("only Q and K are quantised, Q in 128 x d blocks
-// and K in 64 x d blocks, symmetric absmax / 127").
+// Block quantisation ("only Q and K are quantised, Q in 128 x d blocks and K
+// in 64 x d blocks, symmetric absmax / 127").  One launch covers every Q block
+// and every K block; one CTA per (block, head) holds its block in registers
+// (at most eight 16-byte chunks per thread), so HBM sees each fp16 element
+// read once and each code written once.  codes = clamp(rne(x / s), +-127)
+// with s = a / 127, both divisions IEEE fp32.
 // ===================================================================
 constexpr int kQuantThreads = 256;
+constexpr int kQuantChunks = 8;  // per thread: 128 rows x 128 dims / 8 / 256
+
+struct QuantSide {
+  const __half* x;
+  const int32_t* cu_tiles;
+  int8_t* codes;
+  float* scales;
+  int total_tiles, heads, block_rows;
+};
+
+// rne(f / s) without a division on the common path.  y = f * rcp_rn(s) is
+// within 2^-15 of the correctly rounded quotient (|f / s| <= 127, two
+// roundings of 2^-24 relative each), so whenever y lies more than 2^-12 from
+// every half-integer both round to the same integer; inside that band the
+// quotient is taken with the IEEE division itself.
+__device__ __forceinline__ int quant_code(float f, float s, float r) {
+  float y = __fmul_rn(f, r);
+  const float t = fabsf(__fsub_rn(y, rintf(y)));
+  if (fabsf(__fsub_rn(t, 0.5f)) < 0x1p-12f) y = __fdiv_rn(f, s);
+  return max(-127, min(127, __float2int_rn(y)));
+}
 
 __global__ void __launch_bounds__(kQuantThreads)
-    quantize_blocks_kernel(const __half* __restrict__ x, const int32_t* __restrict__ cu_seqlens,
-                           const int32_t* __restrict__ cu_tiles, int nseq, int total_tiles,
-                           int heads, int d, int block_rows, int8_t* __restrict__ codes,
-                           float* __restrict__ scales) {
-  const int tile = blockIdx.x;
-  const int h = blockIdx.y;
-  // sequence that owns this block (few sequences: linear scan)
-  int s = 0;
-  while (s + 1 < nseq && cu_tiles[s + 1] <= tile) ++s;
-  const int t0 = cu_seqlens[s];
-  const int L = cu_seqlens[s + 1] - t0;
-  const int r0 = (tile - cu_tiles[s]) * block_rows;
-  const int rows = min(block_rows, L - r0);
-  const int chunks_per_row = d / 8;  // 16-byte chunks
-  const int nchunks = rows * chunks_per_row;
-
-  float amax = 0.f;
-  for (int c = threadIdx.x; c < nchunks; c += kQuantThreads) {
-    const int r = c / chunks_per_row, cc = c % chunks_per_row;
-    const uint4 u = *reinterpret_cast<const uint4*>(
-        x + (static_cast<size_t>(t0 + r0 + r) * heads + h) * d + cc * 8);
-    const __half2* hv = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __half22float2(hv[k]);
-      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-    }
+    quantize_qk_kernel(QuantSide qs, QuantSide ks, const int32_t* __restrict__ cu_seqlens,
+                       int nseq, int d) {
+  const int nq = qs.total_tiles * qs.heads;
+  const bool is_q = static_cast<int>(blockIdx.x) < nq;
+  // field-wise selection keeps both parameter structs in the constant bank
+  const __half* x = is_q ? qs.x : ks.x;
+  const int32_t* cu_tiles = is_q ? qs.cu_tiles : ks.cu_tiles;
+  int8_t* codes = is_q ? qs.codes : ks.codes;
+  float* scales = is_q ? qs.scales : ks.scales;
+  const int total_tiles = is_q ? qs.total_tiles : ks.total_tiles;
+  const int heads = is_q ? qs.heads : ks.heads;
+  const int block_rows = is_q ? qs.block_rows : ks.block_rows;
+  const int b = is_q ? blockIdx.x : blockIdx.x - nq;
+  const int tile = b / heads;
+  const int h = b - tile * heads;
+  // owning sequence: last s with cu_tiles[s] <= tile
+  int lo = 0, hi = nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu_tiles + mid) <= tile) lo = mid; else hi = mid - 1;
   }
+  const int t0 = __ldg(cu_seqlens + lo);
+  const int L = __ldg(cu_seqlens + lo + 1) - t0;
+  const int r0 = (tile - __ldg(cu_tiles + lo)) * block_rows;
+  const int rows = min(block_rows, L - r0);
+  const int cpr_log2 = d == 128 ? 4 : 3;  // 16-byte chunks per row
+  const int nchunks = rows << cpr_log2;
+  const size_t row_stride = static_cast<size_t>(heads) * d;
+  const size_t base = (static_cast<size_t>(t0 + r0) * heads + h) * d;
+
+  uint4 u[kQuantChunks];
+  __half2 amax2 = __float2half2_rn(0.f);
+#pragma unroll
+  for (int i = 0; i < kQuantChunks; ++i) {
+    const int c = threadIdx.x + i * kQuantThreads;
+    u[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (c < nchunks) {
+      const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
+      u[i] = *reinterpret_cast<const uint4*>(x + off);
+    }
+    const __half2* hv = reinterpret_cast<const __half2*>(&u[i]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) amax2 = __hmax2(amax2, __habs2(hv[k]));
+  }
+  float amax = fmaxf(__low2float(amax2), __high2float(amax2));
   __shared__ float red[kQuantThreads / 32];
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0.f;
+  float a = red[0];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-    if (threadIdx.x == 0) red[0] = v;
-  }
-  __syncthreads();
-  const float a = red[0];
-  const float sc = __fdiv_rn(a, 127.0f);
-  if (threadIdx.x == 0) scales[static_cast<size_t>(h) * total_tiles + tile] = sc;
+  for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
+  const float s = __fdiv_rn(a, 127.0f);
+  if (threadIdx.x == 0) scales[static_cast<size_t>(h) * total_tiles + tile] = s;
+  const float r = a > 0.f ? __frcp_rn(s) : 0.f;
 
-  for (int c = threadIdx.x; c < nchunks; c += kQuantThreads) {
-    const int r = c / chunks_per_row, cc = c % chunks_per_row;
-    const size_t off = (static_cast<size_t>(t0 + r0 + r) * heads + h) * d + cc * 8;
-    const uint4 u = *reinterpret_cast<const uint4*>(x + off);
-    const __half2* hv = reinterpret_cast<const __half2*>(&u);
-    uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __half22float2(hv[k]);
-      int c0 = 0, c1 = 0;
-      if (a > 0.f) {
-        c0 = __float2int_rn(__fdiv_rn(f.x, sc));
-        c1 = __float2int_rn(__fdiv_rn(f.y, sc));
-        c0 = max(-127, min(127, c0));
-        c1 = max(-127, min(127, c1));
+  for (int i = 0; i < kQuantChunks; ++i) {
+    const int c = threadIdx.x + i * kQuantThreads;
+    if (c < nchunks) {
+      const __half2* hv = reinterpret_cast<const __half2*>(&u[i]);
+      uint32_t packed[2];
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const float2 f0 = __half22float2(hv[2 * k2]);
+        const float2 f1 = __half22float2(hv[2 * k2 + 1]);
+        uint32_t w = 0u;
+        if (a > 0.f) {
+          w = (static_cast<uint32_t>(quant_code(f0.x, s, r)) & 0xffu) |
+              ((static_cast<uint32_t>(quant_code(f0.y, s, r)) & 0xffu) << 8) |
+              ((static_cast<uint32_t>(quant_code(f1.x, s, r)) & 0xffu) << 16) |
+              (static_cast<uint32_t>(quant_code(f1.y, s, r)) << 24);
+        }
+        packed[k2] = w;
       }
-      const uint32_t b = (static_cast<uint32_t>(c0) & 0xffu) | ((static_cast<uint32_t>(c1) & 0xffu) << 8);
-      packed[k >> 1] |= b << ((k & 1) * 16);
+      const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
+      *reinterpret_cast<uint2*>(codes + off) = make_uint2(packed[0], packed[1]);
     }
-    *reinterpret_cast<uint2*>(codes + off) = make_uint2(packed[0], packed[1]);
   }
 }
 
-int launch_quantize(const void* x, const int32_t* cu_seqlens, const int32_t* cu_tiles, int nseq,
-                    int total_tiles, int heads, int d, int block_rows, int8_t* codes,
-                    float* scales, cudaStream_t stream) {
-  if (total_tiles == 0 || heads == 0) return cudaSuccess;
-  dim3 grid(total_tiles, heads);
-  quantize_blocks_kernel<<<grid, kQuantThreads, 0, stream>>>(
-      static_cast<const __half*>(x), cu_seqlens, cu_tiles, nseq, total_tiles, heads, d,
-      block_rows, codes, scales);
+int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
+                       const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
+                       int total_qtiles, int total_ktiles, int hq, int hk, int d, int8_t* q8,
+                       float* q_scale, int8_t* k8, float* k_scale, cudaStream_t stream) {
+  QuantSide qs{static_cast<const __half*>(q), cu_qtiles, q8, q_scale, q ? total_qtiles : 0,
+               hq, BM};
+  QuantSide ks{static_cast<const __half*>(k), cu_ktiles, k8, k_scale, k ? total_ktiles : 0,
+               hk, BN};
+  const long long blocks = static_cast<long long>(qs.total_tiles) * hq +
+                           static_cast<long long>(ks.total_tiles) * hk;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  quantize_qk_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+      qs, ks, cu_seqlens, nseq, d);
   return static_cast<int>(cudaGetLastError());
 }
 
