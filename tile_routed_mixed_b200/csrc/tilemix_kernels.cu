@@ -180,7 +180,7 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
 //
 // One CTA per (sequence, query head, pair of query-tile rows 2j and 2j+1),
 // heaviest pairs first.  The two 128-row Q tiles share every K/V tile load.
-// Warp roles (16 warps, four warpgroups):
+// Warp roles (12 warps, three warpgroups):
 //   warp 0      TMA producer: both Q tiles (fp16 and int8), then per key tile
 //               the K tile in each precision the two rows' routing bits need,
 //               and the fp16 V tile
@@ -190,24 +190,17 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
 //               tile q, then O_q += P_q V (kind::f16, P read from TMEM)
 //   warps 4-7   softmax of Q tile 0, warps 8-11 softmax of Q tile 1: one query
 //               row per thread; routed scores -> float score domain, legality
-//               mask, online max / normaliser, P in fp16 back to TMEM; at the
-//               end O / l in fp16
-//   warps 12-15 correction of Q tile 0, warps 16-19 of Q tile 1: when a row's
-//               running max moved, rescale its O accumulator in TMEM (after
-//               the previous P.V landed) before the next P.V is issued, off
-//               the softmax warps' critical path
+//               mask, online max / normaliser, P in fp16 back to TMEM; when a
+//               row's running max moved (rare with lazy rescaling), the warp
+//               rescales its rows of O in TMEM after the previous P.V landed,
+//               before P is handed to the next P.V; at the end O / l in fp16
 // TMEM (512 columns): per Q tile q, O_q [D cols] and two 64-column score
 // buffers, at column offset 256 q.
 // ===================================================================
 constexpr int kStages = 3;
-constexpr int kPrefillThreads = 640;
-constexpr int kCorrectionWarp0 = 12;
-// Register split (setmaxnreg): producer/MMA warpgroup, two softmax
-// warpgroups, two correction warpgroups.  128 * (80 + 2 * 152 + 2 * 48) =
-// 61440 = 640 threads * 96 registers at launch.
-constexpr uint32_t kRegsControl = 80;
-constexpr uint32_t kRegsSoftmax = 152;
-constexpr uint32_t kRegsCorrection = 48;
+constexpr int kPrefillThreads = 384;
+// No register split: every role fits in the registers the launch gives
+// each of the 384 threads.
 constexpr int kSoftmaxWarp0 = 4;
 // Lazy rescaling: the running max used for P is only moved when the tile max
 // exceeds it by more than this (log2 units), so P <= 2^15 stays inside fp16
@@ -229,8 +222,7 @@ struct Smem {
   static constexpr int kOffK8 = kOffK16 + kStages * kK16;  // + stage * kK8
   static constexpr int kOffV = kOffK8 + kStages * kK8;     // + stage * kV
   static constexpr int kOffBar = kOffV + kStages * kV;
-  static constexpr int kOffAlpha = kOffBar + 512;          // float [2][2][128]
-  static constexpr int kBytes = kOffAlpha + 2048 + 1024;    // + alignment slack
+  static constexpr int kBytes = kOffBar + 512 + 1024;      // + alignment slack
   static constexpr int kF16Steps = D / 16;
   static constexpr int kI8Steps = D / 32;
   static constexpr uint32_t kI8Layout = D == 128 ? ptx::kSwizzle128B : ptx::kSwizzle64B;
@@ -249,17 +241,16 @@ struct Smem {
 // s_free(i), which needs the softmax to have read S(i).  P is double-buffered
 // and the softmax stores P(i) only after S(i) landed, whose commit follows
 // P(i-2).V (issued earlier by the same thread), so P(i-2).V has completed:
-// the correction cannot fall two phases behind p_full, and every waiter of
-// pv_done / o_ready is at most one phase behind.
+// the MMA warp cannot fall two phases behind p_full, and the softmax's wait
+// on pv_done for P(i-1).V (before a rescale of O) is at most one phase behind.
 struct Barriers {
   uint64_t q_full;
   uint64_t kv_full[kStages];   // K (both precisions needed) and V of a key tile landed
   uint64_t kv_empty[kStages];  // P.V of that key tile done by every Q tile using it
   uint64_t s_full[2];                   // S_q(i) in TMEM
   uint64_t s_free[2];                   // S_q(i) read out: the S columns may be refilled
-  uint64_t p_full[2][2];                // P_q(j) in TMEM buffer j & 1
+  uint64_t p_full[2][2];                // P_q(j) in TMEM buffer j & 1 (and O_q rescaled)
   uint64_t pv_done[2][2];               // P(j).V of Q tile q done, buffer j & 1
-  uint64_t o_ready[2][2];               // O_q rescaled (if needed) for P(j).V
   uint64_t o_final[2];                  // the last P.V of Q tile q done
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -304,15 +295,6 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity,
       return;
     }
   }
-}
-
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Routing lookup along consecutive key tiles: group = tile / g, tracked
@@ -448,7 +430,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int i = 0; i < 2; ++i) {
         ptx::mbar_init(&bars->p_full[q][i], 128);
         ptx::mbar_init(&bars->pv_done[q][i], 1);
-        ptx::mbar_init(&bars->o_ready[q][i], 128);
       }
       ptx::mbar_init(&bars->o_final[q], 1);
       ptx::mbar_init(&bars->s_full[q], 1);
@@ -470,11 +451,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   volatile int* abort_flag = &bars->abort;
   const unsigned long long tmo = p.timeout_ns;
 
-  float* alpha_smem = reinterpret_cast<float*>(smem + S::kOffAlpha);  // [q][buffer][row]
 
-  if (warp < 4) {
-    regs_dec<kRegsControl>();
-  }
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
@@ -594,7 +571,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               }
             ptx::fence_proxy_async_smem();
           }
-          if (!wait_bar(&bars->o_ready[q][pb], (j >> 1) & 1, abort_flag, tmo)) {
+          if (!wait_bar(&bars->p_full[q][pb], (j >> 1) & 1, abort_flag, tmo)) {
             ok = false;
             break;
           }
@@ -612,9 +589,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       ptx::mma_commit(&bars->drain[q]);
       drain_bar(&bars->drain[q], 0, tmo);
     }
-  } else if (warp >= kSoftmaxWarp0 && warp < kCorrectionWarp0) {
+  } else if (warp >= kSoftmaxWarp0) {
     // ================= softmax / epilogue =================
-    regs_inc<kRegsSoftmax>();
     const int q = (warp - kSoftmaxWarp0) >> 2;        // Q tile of this warpgroup
     const int tr = threadIdx.x - (kSoftmaxWarp0 + 4 * q) * 32;  // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -713,8 +689,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
         m = m_use;
         if (tr == 0) TRACE(15, q, i);
-        // the correction warps rescale O by alpha before P(i).V is issued
-        alpha_smem[(q * 2 + sb) * BM + tr] = (i > 0) ? alpha : 1.0f;
+        if (i > 0 && __any_sync(0xffffffffu, resc)) {
+          // O holds P.V of tiles < i: rescale this warp's rows once P(i-1).V
+          // has landed (rows without a max move multiply by 1)
+          if (!wait_bar_warp(&bars->pv_done[q][(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, tmo)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            const uint32_t to = tmem + lane_base + S::col_o(q) + cc * 32;
+            ptx::tmem_ld32(to, o);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            ptx::tmem_st32(to, o);
+          }
+        }
         // P buffer sb held P(i - 2).  Its P.V was issued before S(i) by the
         // same thread, and the commit that signalled S(i) covers every MMA
         // issued before it, so P(i - 2).V has completed: no wait needed.
@@ -751,41 +744,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           p.lse[static_cast<size_t>(h) * p.total_tokens + t0 + my_row] =
               (m + __log2f(l)) * 0.69314718055994530942f;
       }
-    }
-  } else if (warp >= kCorrectionWarp0) {
-    // ================= correction =================
-    regs_dec<kRegsCorrection>();
-    const int q = (warp - kCorrectionWarp0) >> 2;  // Q tile of this warpgroup
-    const int tr = threadIdx.x - (kCorrectionWarp0 + 4 * q) * 32;  // row within the tile
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int ntq = q ? nt1 : nt0;
-    uint32_t r[32];
-    for (int i = 0; i < ntq; ++i) {
-      const int sb = i & 1;
-      if (!wait_bar_warp(&bars->p_full[q][sb], (i >> 1) & 1, abort_flag, tmo)) break;
-      if (tr == 0) TRACE(2, q, i);
-      const float alpha = alpha_smem[(q * 2 + sb) * BM + tr];
-      if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-        // O_q holds P.V of tiles < i: rescale it once P(i-1).V has landed.
-        if (tr == 0) TRACE(13, q, i);
-        if (!wait_bar_warp(&bars->pv_done[q][(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, tmo))
-          break;
-        if (tr == 0) TRACE(14, q, i);
-        ptx::tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          const uint32_t to = tmem + lane_base + S::col_o(q) + cc * 32;
-          ptx::tmem_ld32(to, r);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-          ptx::tmem_st32(to, r);
-        }
-        ptx::tmem_st_wait();
-      }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->o_ready[q][sb]);
-      if (tr == 0) TRACE(3, q, i);
     }
   }
 
