@@ -31,6 +31,18 @@ __device__ unsigned int g_status;
 // trace[(event * 2 + q) * 256 + tile].
 __device__ unsigned long long* g_trace;
 __device__ int g_trace_cta;
+// Profiling builds only: per CTA [start, set up, -, first epilogue, -, end]
+// in global-timer ns.
+__device__ unsigned long long* g_cta_trace;
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define CTA_TRACE(slot, value)                                                     \
+  do {                                                                             \
+    if (g_cta_trace) g_cta_trace[static_cast<size_t>(blockIdx.x) * 8 + (slot)] = (value); \
+  } while (0)
 #define TRACE(ev, q, i)                                               \
   do {                                                                \
     if (trace_buf && (i) < 256) trace_buf[((ev) * 2 + (q)) * 256 + (i)] = clock64(); \
@@ -38,6 +50,9 @@ __device__ int g_trace_cta;
 #else
 #define TRACE(ev, q, i) \
   do {                  \
+  } while (0)
+#define CTA_TRACE(slot, value) \
+  do {                         \
   } while (0)
 #endif
 
@@ -178,8 +193,11 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
 // ===================================================================
 // Fused attention forward.
 //
-// One CTA per (sequence, query head, pair of query-tile rows 2j and 2j+1),
-// heaviest pairs first.  The two 128-row Q tiles share every K/V tile load.
+// Persistent CTAs, one per SM, each walking a share of the work items: one
+// item per (sequence, query head, pair of query-tile rows 2j and 2j+1),
+// heaviest pairs first.  The two 128-row Q tiles of an item share every K/V
+// tile load; the K/V ring, the score and P buffers run on across items, so
+// one item's last tiles and epilogue overlap the next item's first tiles.
 // Warp roles (12 warps, three warpgroups):
 //   warp 0      TMA producer: both Q tiles (fp16 and int8), then per key tile
 //               the K tile in each precision the two rows' routing bits need,
@@ -236,26 +254,30 @@ struct Smem {
 };
 
 // Every mbarrier below is waited on by parity.  A parity wait is only
-// unambiguous when the waiter is at most one phase behind the barrier, so each
-// barrier is sized so that this holds.  S is single-buffered: S(i+1) needs
-// s_free(i), which needs the softmax to have read S(i).  P is double-buffered
-// and the softmax stores P(i) only after S(i) landed, whose commit follows
-// P(i-2).V (issued earlier by the same thread), so P(i-2).V has completed:
-// the MMA warp cannot fall two phases behind p_full, and the softmax's wait
-// on pv_done for P(i-1).V (before a rescale of O) is at most one phase behind.
+// unambiguous when the waiter is at most one phase behind the barrier; for
+// each wait, the barrier's next phase needs an event that cannot happen before
+// the waiter has moved on (noted at the waits).  The CTA is persistent, so the
+// phases run on across work items: each role keeps running counts.
+//   S is single-buffered: S(n+1) needs s_free(n), i.e. the softmax has read
+//   S(n).  P is double-buffered; the softmax stores P(n) only after S(n)
+//   landed, and the MMA thread issues S(n) after P(n-2).V, so that commit
+//   covers P(n-2).V: the MMA thread cannot fall two phases behind p_full.
 struct Barriers {
-  uint64_t q_full;
-  uint64_t kv_full[kStages];   // K (both precisions needed) and V of a key tile landed
-  uint64_t kv_empty[kStages];  // P.V of that key tile done by every Q tile using it
-  uint64_t s_full[2];                   // S_q(i) in TMEM
-  uint64_t s_free[2];                   // S_q(i) read out: the S columns may be refilled
-  uint64_t p_full[2][2];                // P_q(j) in TMEM buffer j & 1 (and O_q rescaled)
-  uint64_t pv_done[2][2];               // P(j).V of Q tile q done, buffer j & 1
-  uint64_t o_final[2];                  // the last P.V of Q tile q done
+  uint64_t q_full[2];          // Q tile q (fp16 and int8) of the current item landed
+  uint64_t q_free[2];          // the last S = Q K^T of Q tile q's item completed
+  uint64_t kv_full[kStages];   // K (each precision needed) and V of a key tile landed
+  uint64_t kv_empty[kStages];  // both MMA threads are done with that key tile
+  uint64_t s_full[2];          // S_q in TMEM
+  uint64_t s_free[2];          // S_q read out: the S columns may be refilled
+  uint64_t p_full[2][2];       // P_q in TMEM buffer b (and O_q rescaled if needed)
+  uint64_t pv_done[2][2];      // the P.V reading P_q buffer b completed
+  uint64_t o_final[2];         // the last P.V of Q tile q's item completed
+  uint64_t o_free[2];          // the softmax has read O_q of the item out of TMEM
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(Barriers) <= 512, "barrier block exceeds its shared-memory slot");
 
 // Bounded wait: gives up after `timeout_ns` (latching kStatusTimeout and the
 // CTA's abort flag) or as soon as another role of the CTA has given up.
@@ -369,6 +391,59 @@ __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint32_t vb
                     (!first || kk > 0) ? 1u : 0u);
 }
 
+// One work item: query-tile rows 2 pair and 2 pair + 1 (the second may not
+// exist) of sequence s and query head h.  Causal and boundary legality fix
+// each row's key-tile count, independently of the routing words.
+struct WorkItem {
+  int s, h, t0, L, qt0, nt0, nt1, nt, nq, kv, gs, cq, ck;
+  uint64_t w0, w1;
+};
+
+// Decodes item w (heaviest query-tile pairs first, heads innermost).  False
+// if the sequence has no such pair, or if its routing would need a group
+// index above 63 (reported in the status word).
+__device__ __forceinline__ bool load_item(const PrefillParams& p, int w, WorkItem& it) {
+  const int h = w % p.hq;
+  const int s = (w / p.hq) % p.nseq;
+  const int pair = p.max_qpairs - 1 - w / (p.hq * p.nseq);
+  // independent loads first, so that they overlap
+  const int t0 = __ldg(p.cu_seqlens + s);
+  const int t1 = __ldg(p.cu_seqlens + s + 1);
+  const int gs = __ldg(p.g + s);
+  const int cq = __ldg(p.cu_qtiles + s);
+  const int ck = __ldg(p.cu_ktiles + s);
+  const int kv = p.kv_head_of_q ? __ldg(p.kv_head_of_q + h) : h / p.group;
+  const int L = t1 - t0;
+  const int tm = (L + BM - 1) / BM;
+  const int qt0 = 2 * pair;
+  if (qt0 >= tm) return false;
+  const bool has1 = qt0 + 1 < tm;
+  const int nt0 = (p.causal ? min(qt0 * BM + BM, L) - 1 : L - 1) / BN + 1;
+  const int nt1 = has1 ? (p.causal ? min(qt0 * BM + 2 * BM, L) - 1 : L - 1) / BN + 1 : 0;
+  const int nt = max(nt0, nt1);
+  if (gs < 1 || (nt - 1) / gs > 63) {
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusBadGroups);
+    return false;
+  }
+  const uint64_t* wrow = p.masks + static_cast<size_t>(cq + qt0) * p.hk + kv;
+  it.s = s;
+  it.h = h;
+  it.t0 = t0;
+  it.L = L;
+  it.qt0 = qt0;
+  it.nt0 = nt0;
+  it.nt1 = nt1;
+  it.nt = nt;
+  it.nq = has1 ? 2 : 1;
+  it.kv = kv;
+  it.gs = gs;
+  it.cq = cq;
+  it.ck = ck;
+  it.w0 = __ldg(wrow);
+  it.w1 = has1 ? __ldg(wrow + p.hk) : 0ull;
+  return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ PrefillParams p) {
@@ -382,61 +457,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   unsigned long long* const trace_buf =
       static_cast<int>(blockIdx.x) == g_trace_cta ? g_trace : nullptr;
 #endif
-  // A wait of an earlier CTA already expired: do not start more work.
+  if (threadIdx.x == 0) CTA_TRACE(0, gtimer());
+  // A wait of an earlier launch already expired: do not start more work.
   if (*reinterpret_cast<volatile unsigned int*>(&g_status) & kStatusTimeout) return;
-
-  // ---- work item: heaviest query-tile pairs first, heads innermost ----
-  int b = blockIdx.x;
-  const int h = b % p.hq;
-  b /= p.hq;
-  const int s = b % p.nseq;
-  b /= p.nseq;
-  const int pair = p.max_qpairs - 1 - b;
-  const int t0 = p.cu_seqlens[s];
-  const int L = p.cu_seqlens[s + 1] - t0;
-  const int tm = (L + BM - 1) / BM;
-  if (2 * pair >= tm) return;
-  const int kv = p.kv_head_of_q ? p.kv_head_of_q[h] : h / p.group;
-  const int gs = p.g[s];
-  // The CTA's two Q tiles: query-tile rows 2 pair and 2 pair + 1 (the second
-  // may not exist).  Causal and boundary legality fix each row's key-tile
-  // count, independently of the routing words.
-  const int qt0 = 2 * pair;
-  const int last0 = p.causal ? (min(qt0 * BM + BM, L) - 1) / BN : (L - 1) / BN;
-  const int nt0 = last0 + 1;
-  const bool has1 = qt0 + 1 < tm;
-  const int last1 = p.causal ? (min(qt0 * BM + 2 * BM, L) - 1) / BN : (L - 1) / BN;
-  const int nt1 = has1 ? last1 + 1 : 0;
-  const uint64_t* wrow = p.masks + static_cast<size_t>(p.cu_qtiles[s] + qt0) * p.hk + kv;
-  const uint64_t w0 = wrow[0];
-  const uint64_t w1 = has1 ? wrow[p.hk] : 0ull;
-  const int nt = max(nt0, nt1);
-  if (gs < 1 || (nt - 1) / gs > 63) {
-    if (threadIdx.x == 0) atomicOr(&g_status, kStatusBadGroups);
-    return;
-  }
-  const int nq = has1 ? 2 : 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Persistent CTA: in round r the CTAs take the next gridDim.x items of the
+  // heaviest-first order, left to right in even rounds and right to left in
+  // odd ones, which evens out the CTAs' totals; every role walks the same
+  // list.
+  const int num_items = p.max_qpairs * p.nseq * p.hq;
+  const auto item_of_round = [](int rnd) {
+    return rnd * static_cast<int>(gridDim.x) +
+           ((rnd & 1) ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x));
+  };
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&bars->q_full, 1);
     for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(&bars->kv_full[i], 1);
-      ptx::mbar_init(&bars->kv_empty[i], nq);
+      ptx::mbar_init(&bars->kv_empty[i], 2);  // one commit per MMA thread and key tile
     }
     for (int q = 0; q < 2; ++q) {
+      ptx::mbar_init(&bars->q_full[q], 1);
+      ptx::mbar_init(&bars->q_free[q], 1);
       for (int i = 0; i < 2; ++i) {
         ptx::mbar_init(&bars->p_full[q][i], 128);
         ptx::mbar_init(&bars->pv_done[q][i], 1);
       }
       ptx::mbar_init(&bars->o_final[q], 1);
+      ptx::mbar_init(&bars->o_free[q], 128);
       ptx::mbar_init(&bars->s_full[q], 1);
       ptx::mbar_init(&bars->s_free[q], 128);
+      ptx::mbar_init(&bars->drain[q], 1);
     }
-    ptx::mbar_init(&bars->drain[0], 1);
-    ptx::mbar_init(&bars->drain[1], 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -450,141 +504,191 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
   const unsigned long long tmo = p.timeout_ns;
-
+  if (threadIdx.x == 0) CTA_TRACE(1, gtimer());
 
   if (warp == 0) {
     // ================= TMA producer =================
+    // Per item: each Q tile (fp16 and int8) once its slot is free, then per
+    // key tile the K tile in each precision the two rows' routing bits need
+    // and the fp16 V tile, into the 3-stage ring, which runs on across items.
     if (lane == 0) {
+      ptx::prefetch_tensormap(&p.tm_q);
+      ptx::prefetch_tensormap(&p.tm_q8);
       ptx::prefetch_tensormap(&p.tm_k);
       ptx::prefetch_tensormap(&p.tm_k8);
       ptx::prefetch_tensormap(&p.tm_v);
-      ptx::mbar_expect_tx(&bars->q_full, nq * (S::kQ + S::kQ8));
-      for (int q = 0; q < nq; ++q) {
-        const int row = t0 + (qt0 + q) * BM;
-#pragma unroll
-        for (int j = 0; j < D / 64; ++j)
-          ptx::tma_load_3d(smem + S::kOffQ + q * S::kQ + j * BM * 128, &p.tm_q, &bars->q_full,
-                           j * 64, h, row);
-        ptx::tma_load_3d(smem + S::kOffQ8 + q * S::kQ8, &p.tm_q8, &bars->q_full, 0, h, row);
-      }
-      int issued = 0;
-      GroupCursor gc;
-      for (int i = 0; i < nt; ++i, gc.next(gs)) {
-        const int st = i % kStages;
-        // K precisions the two rows need for this tile
-        const bool b0 = gc.int8(w0), b1 = gc.int8(w1);
-        const bool need8 = (i < nt0 && b0) || (i < nt1 && b1);
-        const bool need16 = (i < nt0 && !b0) || (i < nt1 && !b1);
-        if (i >= kStages && !wait_bar(&bars->kv_empty[st], ((i / kStages) - 1) & 1, abort_flag, tmo))
-          break;
-        const int key0 = t0 + i * BN;
-        uint64_t* full = &bars->kv_full[st];
-        ptx::mbar_expect_tx(full, (need16 ? S::kK16 : 0) + (need8 ? S::kK8 : 0) + S::kV);
-        if (need16) {
+      uint32_t kv_tiles = 0;              // key tiles issued so far (ring position)
+      uint32_t q_loads[2] = {0u, 0u};     // loads of each Q slot so far
+      bool ok = true;
+      for (int rnd = 0; ok; ++rnd) {
+        const int w = item_of_round(rnd);
+        if (w >= num_items) break;
+        WorkItem it;
+        if (!load_item(p, w, it)) continue;
+        // Q tile q's slot is refilled once the previous item's last S of it
+        // completed (q_free's next phase needs this load).  Q tile 1 goes
+        // after the item's first key tile, so that the shorter Q tile 0 can
+        // start the item while Q tile 1 still finishes the previous one.
+        const auto load_q = [&](int q) {
+          if (q_loads[q] > 0 &&
+              !wait_bar(&bars->q_free[q], (q_loads[q] - 1) & 1, abort_flag, tmo))
+            return false;
+          const int row = it.t0 + (it.qt0 + q) * BM;
+          ptx::mbar_expect_tx(&bars->q_full[q], S::kQ + S::kQ8);
 #pragma unroll
           for (int j = 0; j < D / 64; ++j)
-            ptx::tma_load_3d(smem + S::kOffK16 + st * S::kK16 + j * BN * 128, &p.tm_k, full,
-                             j * 64, kv, key0);
-        }
-        if (need8)
-          ptx::tma_load_3d(smem + S::kOffK8 + st * S::kK8, &p.tm_k8, full, 0, kv, key0);
+            ptx::tma_load_3d(smem + S::kOffQ + q * S::kQ + j * BM * 128, &p.tm_q,
+                             &bars->q_full[q], j * 64, it.h, row);
+          ptx::tma_load_3d(smem + S::kOffQ8 + q * S::kQ8, &p.tm_q8, &bars->q_full[q], 0, it.h, row);
+          ++q_loads[q];
+          return true;
+        };
+        if (!load_q(0)) break;
+        GroupCursor gc;
+        for (int i = 0; ok && i < it.nt; ++i, gc.next(it.gs)) {
+          const int st = kv_tiles % kStages;
+          // K precisions the two rows need for this tile (at least one: i < nt)
+          const bool b0 = gc.int8(it.w0), b1 = gc.int8(it.w1);
+          const bool need8 = (i < it.nt0 && b0) || (i < it.nt1 && b1);
+          const bool need16 = (i < it.nt0 && !b0) || (i < it.nt1 && !b1);
+          // the stage's previous tile released by both MMA threads
+          if (kv_tiles >= kStages &&
+              !wait_bar(&bars->kv_empty[st], ((kv_tiles / kStages) - 1) & 1, abort_flag, tmo)) {
+            ok = false;
+            break;
+          }
+          const int key0 = it.t0 + i * BN;
+          uint64_t* full = &bars->kv_full[st];
+          ptx::mbar_expect_tx(full, (need16 ? S::kK16 : 0) + (need8 ? S::kK8 : 0) + S::kV);
+          if (need16) {
 #pragma unroll
-        for (int j = 0; j < D / 64; ++j)
-          ptx::tma_load_3d(smem + S::kOffV + st * S::kV + j * BN * 128, &p.tm_v, full, j * 64, kv,
-                           key0);
-        ++issued;
+            for (int j = 0; j < D / 64; ++j)
+              ptx::tma_load_3d(smem + S::kOffK16 + st * S::kK16 + j * BN * 128, &p.tm_k, full,
+                               j * 64, it.kv, key0);
+          }
+          if (need8)
+            ptx::tma_load_3d(smem + S::kOffK8 + st * S::kK8, &p.tm_k8, full, 0, it.kv, key0);
+#pragma unroll
+          for (int j = 0; j < D / 64; ++j)
+            ptx::tma_load_3d(smem + S::kOffV + st * S::kV + j * BN * 128, &p.tm_v, full, j * 64,
+                             it.kv, key0);
+          ++kv_tiles;
+          if (i == 0 && it.nq == 2 && !load_q(1)) ok = false;
+        }
       }
       // Never leave with copies into this CTA's shared memory in flight.
-      drain_bar(&bars->q_full, 0, tmo);
-      for (int st = 0; st < kStages && st < issued; ++st)
-        drain_bar(&bars->kv_full[st], ((issued - 1 - st) / kStages) & 1, tmo);
+      for (int q = 0; q < 2; ++q)
+        if (q_loads[q] > 0) drain_bar(&bars->q_full[q], (q_loads[q] - 1) & 1, tmo);
+      for (uint32_t st = 0; st < kStages && st < kv_tiles; ++st)
+        drain_bar(&bars->kv_full[st], ((kv_tiles - 1 - st) / kStages) & 1, tmo);
     }
   } else if (warp == 1 || warp == 2) {
     // ================= MMA issuers: warp 1 for Q tile 0, warp 2 for Q tile 1 =====
-    // Order: S_q(0), then per key tile j: S_q(j + 1) as soon as the softmax has
-    // read S_q(j) out of TMEM, then P_q(j).V once O_q is ready for it.  A thread whose Q tile is shorter (or absent) still releases
-    // the remaining K/V stages, after they are loaded, so that each stage's
-    // release barrier sees one arrival per Q tile.
+    // Per item, in key-tile order: S_q(0), then per key tile j: S_q(j + 1) as
+    // soon as the softmax has read S_q(j) out of TMEM, then P_q(j).V once the
+    // softmax has posted P_q(j).  Each thread releases every key tile of every
+    // item (count 2 per stage): after its P.V, or once the tile has landed if
+    // its Q tile does not use it (so that the arrival cannot count towards
+    // the stage's previous tile).
     const int q = warp - 1;
-    if (lane == 0 && q < nq) {
+    if (lane == 0) {
       const uint32_t a_smem = ptx::smem_addr(smem);
       const uint64_t t16 = ptx::smem_desc(0, 16, 1024, ptx::kSwizzle128B);
       const uint64_t t8 = ptx::smem_desc(0, 16, S::kI8Sbo, S::kI8Layout);
       const uint64_t tv = ptx::smem_desc(0, BN * 128, 1024, ptx::kSwizzle128B);
-      const int ntq = q ? nt1 : nt0;
-      const uint64_t word = q ? w1 : w0;
       const uint32_t aq16 = a_smem + S::kOffQ + q * S::kQ;
       const uint32_t aq8 = a_smem + S::kOffQ8 + q * S::kQ8;
       const uint32_t d_o = tmem + S::col_o(q);
-      bool ok = wait_bar(&bars->q_full, 0, abort_flag, tmo);
-      ptx::tc_fence_after();
       const uint32_t d_s = tmem + S::col_s(q);
-      // Every K/V stage of tiles 0 .. nt-1 is awaited exactly once, in order:
-      // before S(i) for tiles this Q tile uses, before the release otherwise.
-#define TILEMIX_KV_WAIT(i) \
-  wait_bar(&bars->kv_full[(i) % kStages], ((i) / kStages) & 1, abort_flag, tmo)
-      GroupCursor gc;  // routing group of the next score tile
-      if (ntq > 0) {
-        if (!TILEMIX_KV_WAIT(0)) ok = false;
-        if (ok) {
-          ptx::tc_fence_after();
-          issue_qk<D>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16, a_smem + S::kOffK8,
-                      t16, t8);
-          ptx::mma_commit(&bars->s_full[q]);
-          TRACE(4, q, 0);
-        }
-        gc.next(gs);
-      }
-      for (int j = 0; ok && j < nt; ++j) {
-        const int st = j % kStages;
-        const int i = j + 1;  // next score tile
-        if (i < ntq) {
-          // S(i) overwrites S(j) once the softmax has read it out
-          if (!wait_bar(&bars->s_free[q], j & 1, abort_flag, tmo) || !TILEMIX_KV_WAIT(i)) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-          const int sti = i % kStages;
-          issue_qk<D>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16 + sti * S::kK16,
-                      a_smem + S::kOffK8 + sti * S::kK8, t16, t8);
-          ptx::mma_commit(&bars->s_full[q]);
-          gc.next(gs);
-          TRACE(4, q, i);
-        } else if (i < nt && !TILEMIX_KV_WAIT(i)) {
+      uint32_t kv_tiles = 0;  // key tiles of earlier items (ring position)
+      uint32_t n_s = 0;       // S_q issued so far
+      uint32_t n_p = 0;       // P_q.V issued so far
+      uint32_t n_items = 0;   // items that had a Q tile q
+      bool ok = true;
+      for (int rnd = 0; ok; ++rnd) {
+        const int w = item_of_round(rnd);
+        if (w >= num_items) break;
+        WorkItem it;
+        if (!load_item(p, w, it)) continue;
+        const bool mine = q < it.nq;
+        const int ntq = !mine ? 0 : (q ? it.nt1 : it.nt0);
+        const uint64_t word = q ? it.w1 : it.w0;
+        // q_full's next phase needs this item's last S, issued below
+        if (mine && !wait_bar(&bars->q_full[q], n_items & 1, abort_flag, tmo)) {
           ok = false;
           break;
         }
-        if (j < ntq) {
-          const int pb = j & 1;
-          const int valid = L - j * BN;
-          if (valid < BN) {
-            // Keys past the sequence end belong to the next packed sequence:
-            // zero their V rows so that 0 * (NaN or Inf) cannot reach O.  The
-            // Q tiles write the same zeros, each before its own P.V.
-            uint8_t* vslot = smem + S::kOffV + st * S::kV;
-            for (int part = 0; part < D / 64; ++part)
-              for (int r = valid; r < BN; ++r) {
-                uint4* row = reinterpret_cast<uint4*>(vslot + part * BN * 128 + r * 128);
+        GroupCursor gc;  // routing group of tile i
+        for (int i = 0; i <= it.nt; ++i) {
+          if (i < it.nt) {
+            const uint32_t t = kv_tiles + i;
+            // S(n) overwrites S(n - 1) once the softmax has read it out
+            if (i < ntq && n_s > 0 && !wait_bar(&bars->s_free[q], (n_s - 1) & 1, abort_flag, tmo)) {
+              ok = false;
+              break;
+            }
+            if (!wait_bar(&bars->kv_full[t % kStages], (t / kStages) & 1, abort_flag, tmo)) {
+              ok = false;
+              break;
+            }
+            if (i < ntq) {
+              ptx::tc_fence_after();
+              const int st = t % kStages;
+              issue_qk<D>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16 + st * S::kK16,
+                          a_smem + S::kOffK8 + st * S::kK8, t16, t8);
+              ptx::mma_commit(&bars->s_full[q]);
+              ++n_s;
+              if (i == ntq - 1) ptx::mma_commit(&bars->q_free[q]);
+              TRACE(4, q, i);
+            }
+            gc.next(it.gs);
+          }
+          if (i >= 1) {
+            const int j = i - 1;
+            const int st = (kv_tiles + j) % kStages;
+            if (j < ntq) {
+              const int valid = it.L - j * BN;
+              if (valid < BN) {
+                // Keys past the sequence end belong to the next packed
+                // sequence: zero their V rows so that 0 * (NaN or Inf) cannot
+                // reach O.  Both Q tiles write the same zeros, each before its
+                // own P.V.
+                uint8_t* vslot = smem + S::kOffV + st * S::kV;
+                for (int part = 0; part < D / 64; ++part)
+                  for (int r = valid; r < BN; ++r) {
+                    uint4* row = reinterpret_cast<uint4*>(vslot + part * BN * 128 + r * 128);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+                    for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+                  }
+                ptx::fence_proxy_async_smem();
               }
-            ptx::fence_proxy_async_smem();
+              // the first P.V of an item overwrites O_q: the previous item's
+              // epilogue must have read it (o_free's next phase needs this
+              // item's o_final)
+              if (j == 0 && n_items > 0 &&
+                  !wait_bar(&bars->o_free[q], (n_items - 1) & 1, abort_flag, tmo)) {
+                ok = false;
+                break;
+              }
+              const int pb = n_p & 1;
+              if (!wait_bar(&bars->p_full[q][pb], (n_p >> 1) & 1, abort_flag, tmo)) {
+                ok = false;
+                break;
+              }
+              TRACE(10, q, j);
+              ptx::tc_fence_after();
+              issue_pv<D>(d_o, tmem + S::col_p(q, pb), a_smem + S::kOffV + st * S::kV, tv, j == 0);
+              ptx::mma_commit(&bars->pv_done[q][pb]);
+              ++n_p;
+              if (j == ntq - 1) ptx::mma_commit(&bars->o_final[q]);
+              TRACE(5, q, j);
+            }
+            ptx::mma_commit(&bars->kv_empty[st]);
           }
-          if (!wait_bar(&bars->p_full[q][pb], (j >> 1) & 1, abort_flag, tmo)) {
-            ok = false;
-            break;
-          }
-          TRACE(10, q, j);
-          ptx::tc_fence_after();
-          issue_pv<D>(d_o, tmem + S::col_p(q, pb), a_smem + S::kOffV + st * S::kV, tv, j == 0);
-          ptx::mma_commit(&bars->pv_done[q][pb]);
-          if (j == ntq - 1) ptx::mma_commit(&bars->o_final[q]);
-          TRACE(5, q, j);
         }
-        ptx::mma_commit(&bars->kv_empty[st]);
+        kv_tiles += it.nt;
+        if (mine) ++n_items;
       }
-#undef TILEMIX_KV_WAIT
       // all MMAs of this thread complete before TMEM and shared memory go away
       ptx::mma_commit(&bars->drain[q]);
       drain_bar(&bars->drain[q], 0, tmo);
@@ -594,26 +698,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int q = (warp - kSoftmaxWarp0) >> 2;        // Q tile of this warpgroup
     const int tr = threadIdx.x - (kSoftmaxWarp0 + 4 * q) * 32;  // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int ntq = q ? nt1 : nt0;
-    const uint64_t word = q ? w1 : w0;
-    const int row0 = (qt0 + q) * BM;
-    const int my_row = row0 + tr;
-    if (ntq > 0) {
-      const float q_sc =
-          p.q_scale[static_cast<size_t>(h) * p.total_qtiles + p.cu_qtiles[s] + qt0 + q];
-      const float* ks = p.k_scale + static_cast<size_t>(kv) * p.total_ktiles + p.cu_ktiles[s];
+    uint32_t n_s = 0;      // S_q read so far
+    uint32_t n_p = 0;      // P_q stored so far
+    uint32_t n_items = 0;  // items that had a Q tile q
+    bool ok = true;
+    uint32_t r[64];
+    for (int rnd = 0; ok; ++rnd) {
+      const int w = item_of_round(rnd);
+      if (w >= num_items) break;
+      WorkItem it;
+      if (!load_item(p, w, it)) continue;
+      if (q >= it.nq) continue;
+      const int h = it.h, s = it.s, kv = it.kv, t0 = it.t0, L = it.L, gs = it.gs;
+      const int ntq = q ? it.nt1 : it.nt0;
+      const uint64_t word = q ? it.w1 : it.w0;
+      const int row0 = (it.qt0 + q) * BM;
+      const int my_row = row0 + tr;
+      const float q_sc = __ldg(p.q_scale + static_cast<size_t>(h) * p.total_qtiles + it.cq + it.qt0 + q);
+      const float* ks = p.k_scale + static_cast<size_t>(kv) * p.total_ktiles + it.ck;
+      (void)s;
       float m = -INFINITY;  // running max, log2 units
       float l = 0.f;        // normaliser: sum of the fp16-rounded P actually used in P.V
-      bool ok = true;
-      uint32_t r[64];
       float k_sc_next = __ldg(ks);
       GroupCursor gc;
       for (int i = 0; i < ntq; ++i, gc.next(gs)) {
-        const int sb = i & 1;
+        const int sb = n_p & 1;
         const bool is_int = gc.int8(word);
         const float k_sc = k_sc_next;
         if (i + 1 < ntq) k_sc_next = __ldg(ks + i + 1);
-        if (!wait_bar_warp(&bars->s_full[q], i & 1, abort_flag, tmo)) {
+        // s_full's next phase needs s_free from this read
+        if (!wait_bar_warp(&bars->s_full[q], n_s & 1, abort_flag, tmo)) {
           ok = false;
           break;
         }
@@ -623,9 +737,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ptx::tmem_ld32(ts, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         ptx::tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         ptx::tmem_ld_wait();
-        // S(i) is in registers: the MMA warp may compute S(i + 1) now
+        // S is in registers: the MMA warp may compute the next S now
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->s_free[q]);
+        ++n_s;
         if (tr == 0) TRACE(11, q, i);
         if (is_int && p.dbg && my_row < L) {
           int32_t* drow =
@@ -692,7 +807,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (i > 0 && __any_sync(0xffffffffu, resc)) {
           // O holds P.V of tiles < i: rescale this warp's rows once P(i-1).V
           // has landed (rows without a max move multiply by 1)
-          if (!wait_bar_warp(&bars->pv_done[q][(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, tmo)) {
+          // (the P.V of the previous tile is the (n_p - 1)-th; the next phase
+          // of its pv_done barrier needs p_full from this tile)
+          if (!wait_bar_warp(&bars->pv_done[q][(n_p - 1) & 1], ((n_p - 1) >> 1) & 1, abort_flag, tmo)) {
             ok = false;
             break;
           }
@@ -708,42 +825,52 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             ptx::tmem_st32(to, o);
           }
         }
-        // P buffer sb held P(i - 2).  Its P.V was issued before S(i) by the
-        // same thread, and the commit that signalled S(i) covers every MMA
-        // issued before it, so P(i - 2).V has completed: no wait needed.
+        // P buffer sb held the P stored two tiles ago.  Its P.V was issued
+        // before this tile's S by the same thread, and the commit that
+        // signalled S covers every MMA issued before it: no wait needed.
         ptx::tmem_st32(tmem + lane_base + S::col_p(q, sb),
                        *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[q][sb]);
+        ++n_p;
         if (tr == 0) TRACE(1, q, i);
       }
-      if (ok && wait_bar_warp(&bars->o_final[q], 0, abort_flag, tmo)) {
-        ptx::tc_fence_after();
-        const float inv_l = 1.0f / l;
-        const bool valid = my_row < L;
-        __half* orow = static_cast<__half*>(p.o) +
-                       (static_cast<size_t>(t0 + my_row) * p.hq + h) * D;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          ptx::tmem_ld32(tmem + lane_base + S::col_o(q) + cc * 32,
-                         *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            r[32 + j] = pack_f16x2(__uint_as_float(r[2 * j]) * inv_l,
-                                   __uint_as_float(r[2 * j + 1]) * inv_l);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(r[32 + 4 * j], r[33 + 4 * j], r[34 + 4 * j], r[35 + 4 * j]);
-          }
-        }
-        if (p.lse && valid)
-          p.lse[static_cast<size_t>(h) * p.total_tokens + t0 + my_row] =
-              (m + __log2f(l)) * 0.69314718055994530942f;
+      // o_final's next phase needs o_free from this epilogue
+      if (!ok || !wait_bar_warp(&bars->o_final[q], n_items & 1, abort_flag, tmo)) {
+        ok = false;
+        break;
       }
+      if (tr == 0 && q == 0 && rnd == 0) CTA_TRACE(3, gtimer());
+      ptx::tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const bool valid = my_row < L;
+      __half* orow = static_cast<__half*>(p.o) + (static_cast<size_t>(t0 + my_row) * p.hq + h) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        ptx::tmem_ld32(tmem + lane_base + S::col_o(q) + cc * 32,
+                       *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        ptx::tmem_ld_wait();
+        if (cc == D / 32 - 1) {
+          // O_q is in registers: the next item's first P.V may overwrite it
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&bars->o_free[q]);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          r[32 + j] = pack_f16x2(__uint_as_float(r[2 * j]) * inv_l,
+                                 __uint_as_float(r[2 * j + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(r[32 + 4 * j], r[33 + 4 * j], r[34 + 4 * j], r[35 + 4 * j]);
+        }
+      }
+      if (p.lse && valid)
+        p.lse[static_cast<size_t>(h) * p.total_tokens + t0 + my_row] =
+            (m + __log2f(l)) * 0.69314718055994530942f;
+      ++n_items;
     }
   }
 
@@ -753,6 +880,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
+  if (threadIdx.x == 0) CTA_TRACE(5, gtimer());
 }
 
 template <int D>
@@ -761,10 +889,17 @@ static int launch_prefill_d(const PrefillParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return static_cast<int>(e);
-  const long long blocks = static_cast<long long>(p.max_qpairs) * p.nseq * p.hq;
-  if (blocks == 0) return cudaSuccess;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  prefill_fwd_kernel<D><<<static_cast<unsigned>(blocks), kPrefillThreads, smem, stream>>>(p);
+  const long long items = static_cast<long long>(p.max_qpairs) * p.nseq * p.hq;
+  if (items == 0) return cudaSuccess;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  // persistent: one CTA per SM (the shared memory admits one), each walking
+  // every gridDim.x-th work item
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return static_cast<int>(e);
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return static_cast<int>(e);
+  const unsigned blocks = static_cast<unsigned>(items < sms ? items : sms);
+  prefill_fwd_kernel<D><<<blocks, kPrefillThreads, smem, stream>>>(p);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -779,6 +914,10 @@ extern "C" TILEMIX_API int tilemix_trace_setup(void* buf, int cta) {
   unsigned long long* ptr = static_cast<unsigned long long*>(buf);
   if (cudaMemcpyToSymbol(g_trace, &ptr, sizeof(ptr)) != cudaSuccess) return 1;
   return cudaMemcpyToSymbol(g_trace_cta, &cta, sizeof(cta)) != cudaSuccess;
+}
+extern "C" TILEMIX_API int tilemix_trace_ctas(void* buf) {
+  unsigned long long* ptr = static_cast<unsigned long long*>(buf);
+  return cudaMemcpyToSymbol(g_cta_trace, &ptr, sizeof(ptr)) != cudaSuccess;
 }
 #endif
 
