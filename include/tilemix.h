@@ -169,15 +169,18 @@ typedef struct tilemix_prefill_args {
 } tilemix_prefill_args;
 
 /* Bytes of device workspace tilemix_prefill_fwd needs for these arguments
- * (it holds the INT8 codes and scales of Q, and of K unless k_i8 is given).
+ * (it holds the INT8 codes and scales of Q, and of K unless k_i8 is given,
+ * and the fused kernel's work-item counter, so calls that may run at the same
+ * time on different streams need separate workspaces).
  * INVALID_ARG on a NULL argument. */
 int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes);
 
 /* Fused tile-routed mixed-precision causal prefill attention forward:
  * O[t, h] = softmax over legal keys of the routed scores, times V, in fp16
  * (one rounding of the fp32 accumulator divided by the normaliser).
- * Enqueues the K quantisation pre-pass (unless k_i8 is given), the Q
- * quantisation and the fused attention kernel on `stream`. */
+ * Enqueues one quantisation launch (Q, and K unless k_i8 is given) and the
+ * fused attention kernel (persistent: one CTA per SM, work items handed out
+ * heaviest first through a counter in the workspace) on `stream`. */
 int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
 
 /* Allocation-free variant of tilemix_prefill_fwd.  (The TileMix pages have no
@@ -189,8 +192,9 @@ int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
  * path where an allocation, which may synchronise the device, is not allowed.
  * The caller still passes q, k, v, o (and the other tensors) as for
  * tilemix_prefill_fwd; args->workspace and args->workspace_bytes are ignored.
- * The INT8 codes and scales that tilemix_prefill_fwd keeps in the caller's
- * workspace live instead in one fixed scratch array of 64 MiB inside the
+ * The INT8 codes and scales (and the work-item counter) that
+ * tilemix_prefill_fwd keeps in the caller's workspace live instead in one
+ * fixed scratch array of 64 MiB inside the
  * library (TILEMIX_NOALLOC_SCRATCH_BYTES), which every GPU that loads the
  * library holds until the process exits.  A call whose workspace would exceed
  * it (tilemix_workspace_size() > 64 MiB) returns TILEMIX_ERR_TOO_LARGE and

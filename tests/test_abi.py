@@ -112,11 +112,12 @@ def test_prefill_argument_checks_are_synchronous():
     L = tm.lib()
     n = ctypes.c_size_t(0)
     assert L.tilemix_workspace_size(ctypes.byref(_fake_args()), ctypes.byref(n)) == tm.OK
-    # q8 [256*4*128] + q scales [4*2 floats] + k8 [256*2*128] + k scales, each 256-aligned
-    assert n.value == 131072 + 256 + 65536 + 256
+    # q8 [256*4*128] + q scales [4*2 floats] + k8 [256*2*128] + k scales, each 256-aligned,
+    # + 256 bytes for the fused kernel's work-item ticket
+    assert n.value == 131072 + 256 + 65536 + 256 + 256
     assert L.tilemix_workspace_size(ctypes.byref(_fake_args(k_i8=4096, k_scale=4096)),
                                     ctypes.byref(n)) == tm.OK
-    assert n.value == 131072 + 256
+    assert n.value == 131072 + 256 + 256
     cases = [
         (dict(d=96), tm.ERR_UNSUPPORTED),
         (dict(hq=3, hk=2), tm.ERR_INVALID_ARG),

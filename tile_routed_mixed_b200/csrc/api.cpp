@@ -67,7 +67,7 @@ int encode_rows(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, i
 }
 
 struct WorkspaceLayout {
-  size_t q8, q_scale, k8, k_scale, total;
+  size_t q8, q_scale, k8, k_scale, ticket, total;
 };
 
 WorkspaceLayout layout_of(const tilemix_prefill_args* a) {
@@ -83,6 +83,8 @@ WorkspaceLayout layout_of(const tilemix_prefill_args* a) {
   if (own_k) off = round_up(off + T * a->hk * a->d, 256);
   w.k_scale = off;
   if (own_k) off = round_up(off + sizeof(float) * a->hk * static_cast<size_t>(a->total_ktiles), 256);
+  w.ticket = off;  // work-item counter of the fused kernel
+  off += 256;
   w.total = off;
   return w;
 }
@@ -105,6 +107,37 @@ int check_args(const tilemix_prefill_args* a) {
       (a->k_i8 && !aligned16(a->k_i8)))
     return TILEMIX_ERR_INVALID_ARG;
   if (a->max_seqlen < 1) return TILEMIX_ERR_INVALID_ARG;
+  return TILEMIX_OK;
+}
+
+// Quantisation of the INT8 operands; a non-null ticket is zeroed by the
+// same launch.
+int quantize_impl(const void* q_f16, const void* k_f16,
+                                    const int32_t* cu_seqlens_d, const int32_t* cu_qtiles_d,
+                                    const int32_t* cu_ktiles_d, int nseq, int total_tokens,
+                                    int total_qtiles, int total_ktiles, int hq, int hk, int d,
+                                    int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                                    int* ticket, void* stream) {
+  if (d != 64 && d != 128) return TILEMIX_ERR_UNSUPPORTED;
+  if (nseq < 0 || total_tokens < 0 || total_qtiles < 0 || total_ktiles < 0)
+    return TILEMIX_ERR_INVALID_ARG;
+  if (nseq == 0 || total_tokens == 0) return TILEMIX_OK;
+  if (!cu_seqlens_d) return TILEMIX_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (q_f16) {
+    if (hq < 1 || !cu_qtiles_d || !q_i8 || !q_scale || !aligned16(q_f16) ||
+        (reinterpret_cast<uintptr_t>(q_i8) & 7u))
+      return TILEMIX_ERR_INVALID_ARG;
+  }
+  if (k_f16) {
+    if (hk < 1 || !cu_ktiles_d || !k_i8 || !k_scale || !aligned16(k_f16) ||
+        (reinterpret_cast<uintptr_t>(k_i8) & 7u))
+      return TILEMIX_ERR_INVALID_ARG;
+  }
+  if (tilemix::launch_quantize_qk(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq,
+                                  total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8,
+                                  k_scale, ticket, st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
   return TILEMIX_OK;
 }
 
@@ -134,27 +167,9 @@ TILEMIX_API int tilemix_quantize_qk(const void* q_f16, const void* k_f16,
                                     int total_qtiles, int total_ktiles, int hq, int hk, int d,
                                     int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
                                     void* stream) {
-  if (d != 64 && d != 128) return TILEMIX_ERR_UNSUPPORTED;
-  if (nseq < 0 || total_tokens < 0 || total_qtiles < 0 || total_ktiles < 0)
-    return TILEMIX_ERR_INVALID_ARG;
-  if (nseq == 0 || total_tokens == 0) return TILEMIX_OK;
-  if (!cu_seqlens_d) return TILEMIX_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (q_f16) {
-    if (hq < 1 || !cu_qtiles_d || !q_i8 || !q_scale || !aligned16(q_f16) ||
-        (reinterpret_cast<uintptr_t>(q_i8) & 7u))
-      return TILEMIX_ERR_INVALID_ARG;
-  }
-  if (k_f16) {
-    if (hk < 1 || !cu_ktiles_d || !k_i8 || !k_scale || !aligned16(k_f16) ||
-        (reinterpret_cast<uintptr_t>(k_i8) & 7u))
-      return TILEMIX_ERR_INVALID_ARG;
-  }
-  if (tilemix::launch_quantize_qk(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq,
-                                  total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8,
-                                  k_scale, st) != cudaSuccess)
-    return TILEMIX_ERR_CUDA;
-  return TILEMIX_OK;
+  return quantize_impl(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq, total_tokens,
+                       total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8, k_scale,
+                       nullptr, stream);
 }
 
 TILEMIX_API int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes) {
@@ -181,10 +196,11 @@ TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream)
   const float* k_scale = a->k_i8 ? a->k_scale : reinterpret_cast<float*>(ws + w.k_scale);
 
   // INT8 path operands: Q always, K unless the caller supplied its codes.
-  rc = tilemix_quantize_qk(a->q, a->k_i8 ? nullptr : a->k, a->cu_seqlens, a->cu_qtiles,
-                           a->cu_ktiles, a->nseq, a->total_tokens, a->total_qtiles,
-                           a->total_ktiles, a->hq, a->hk, a->d, q8, q_scale,
-                           const_cast<int8_t*>(k8), const_cast<float*>(k_scale), stream);
+  int* ticket = reinterpret_cast<int*>(ws + w.ticket);
+  rc = quantize_impl(a->q, a->k_i8 ? nullptr : a->k, a->cu_seqlens, a->cu_qtiles, a->cu_ktiles,
+                     a->nseq, a->total_tokens, a->total_qtiles, a->total_ktiles, a->hq, a->hk,
+                     a->d, q8, q_scale, const_cast<int8_t*>(k8), const_cast<float*>(k_scale),
+                     ticket, stream);
   if (rc != TILEMIX_OK) return rc;
 
   tilemix::PrefillParams p;
@@ -218,6 +234,7 @@ TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream)
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.dbg = a->debug_int32_scores;
+  p.ticket = ticket;
   p.dbg_cols = (a->max_seqlen + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N * TILEMIX_BLOCK_N;
   p.nseq = a->nseq;
   p.total_tokens = T;

@@ -34,6 +34,7 @@ struct PrefillParams {
   const float* q_scale;   // [hq][total_qtiles]
   const float* k_scale;   // [hk][total_ktiles]
   int32_t* dbg;
+  int* ticket;            // work-item ticket, zero at launch (see launch_quantize_qk)
   int dbg_cols;
   int nseq, total_tokens, total_qtiles, total_ktiles, max_qpairs;
   int hq, hk, group;      // group = hq / hk
@@ -44,11 +45,13 @@ struct PrefillParams {
 
 // Launchers implemented in the CUDA translation unit.  Return cudaError_t.
 // One launch quantises Q (128-row blocks) and K (64-row blocks); a null q or
-// k skips that side.
+// k skips that side.  A non-null ticket is set to zero by the same launch
+// (the fused kernel that follows on the stream hands out work from it).
 int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
                        int total_qtiles, int total_ktiles, int hq, int hk, int d, int8_t* q8,
-                       float* q_scale, int8_t* k8, float* k_scale, cudaStream_t stream);
+                       float* q_scale, int8_t* k8, float* k_scale, int* ticket,
+                       cudaStream_t stream);
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
 int read_and_clear_status(unsigned int* status, cudaStream_t stream);
 // Device address of the allocation-free entry point's scratch array on the

@@ -92,7 +92,8 @@ __device__ __forceinline__ int quant_code(float f, float s, float r) {
 
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_qk_kernel(QuantSide qs, QuantSide ks, const int32_t* __restrict__ cu_seqlens,
-                       int nseq, int d) {
+                       int nseq, int d, int* ticket) {
+  if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;
   const int nq = qs.total_tiles * qs.heads;
   const bool is_q = static_cast<int>(blockIdx.x) < nq;
   // field-wise selection keeps both parameter structs in the constant bank
@@ -176,17 +177,19 @@ __global__ void __launch_bounds__(kQuantThreads)
 int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
                        int total_qtiles, int total_ktiles, int hq, int hk, int d, int8_t* q8,
-                       float* q_scale, int8_t* k8, float* k_scale, cudaStream_t stream) {
+                       float* q_scale, int8_t* k8, float* k_scale, int* ticket,
+                       cudaStream_t stream) {
   QuantSide qs{static_cast<const __half*>(q), cu_qtiles, q8, q_scale, q ? total_qtiles : 0,
                hq, BM};
   QuantSide ks{static_cast<const __half*>(k), cu_ktiles, k8, k_scale, k ? total_ktiles : 0,
                hk, BN};
   const long long blocks = static_cast<long long>(qs.total_tiles) * hq +
                            static_cast<long long>(ks.total_tiles) * hk;
-  if (blocks == 0) return cudaSuccess;
+  if (blocks == 0)
+    return ticket ? static_cast<int>(cudaMemsetAsync(ticket, 0, sizeof(int), stream)) : cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   quantize_qk_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-      qs, ks, cu_seqlens, nseq, d);
+      qs, ks, cu_seqlens, nseq, d, ticket);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -274,10 +277,19 @@ struct Barriers {
   uint64_t o_final[2];         // the last P.V of Q tile q's item completed
   uint64_t o_free[2];          // the softmax has read O_q of the item out of TMEM
   uint64_t drain[2];
+  uint64_t item_full[4];       // a work item index published in ring slot k % 4
+  uint64_t item_empty[4];      // every consumer has read ring slot k % 4
+  int item_ring[4];            // item indices, -1 = no more work
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Barriers) <= 512, "barrier block exceeds its shared-memory slot");
+
+// The producer thread takes work items from a global ticket (heaviest first,
+// so faster SMs simply take more) and publishes them through a small ring;
+// both MMA threads and all 256 softmax threads read every slot.
+constexpr int kItemSlots = 4;
+constexpr int kItemConsumers = 2 + 2 * 128;
 
 // Bounded wait: gives up after `timeout_ns` (latching kStatusTimeout and the
 // CTA's abort flag) or as soon as another role of the CTA has given up.
@@ -308,6 +320,22 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity,
 }
 
 // Drain wait used on the way out: ignores the abort flag, still bounded.
+// A consumer's next work item from ring slot k % 4 (item_full's next phase
+// for the slot needs this consumer's item_empty arrival): the index, -1 when
+// there is no more work, or kItemAbort if the wait gave up.
+constexpr int kItemAbort = -2;
+__device__ __forceinline__ int next_item(Barriers* bars, uint32_t k, volatile int* abort_flag,
+                                         unsigned long long tmo, bool warp_wide) {
+  const int slot = k % kItemSlots;
+  const uint32_t parity = (k / kItemSlots) & 1;
+  const bool ok = warp_wide ? wait_bar_warp(&bars->item_full[slot], parity, abort_flag, tmo)
+                            : wait_bar(&bars->item_full[slot], parity, abort_flag, tmo);
+  if (!ok) return kItemAbort;
+  const int w = *reinterpret_cast<volatile int*>(&bars->item_ring[slot]);
+  ptx::mbar_arrive(&bars->item_empty[slot]);  // release: the read above comes first
+  return w;
+}
+
 __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity,
                                           unsigned long long timeout_ns) {
   const unsigned long long start = ptx::globaltimer();
@@ -463,15 +491,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Persistent CTA: in round r the CTAs take the next gridDim.x items of the
-  // heaviest-first order, left to right in even rounds and right to left in
-  // odd ones, which evens out the CTAs' totals; every role walks the same
-  // list.
+  // Persistent CTA: the first item is blockIdx.x, every later one comes from
+  // the ticket (gridDim.x + ticket), in the heaviest-first order.
   const int num_items = p.max_qpairs * p.nseq * p.hq;
-  const auto item_of_round = [](int rnd) {
-    return rnd * static_cast<int>(gridDim.x) +
-           ((rnd & 1) ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x));
-  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -490,6 +512,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       ptx::mbar_init(&bars->s_full[q], 1);
       ptx::mbar_init(&bars->s_free[q], 128);
       ptx::mbar_init(&bars->drain[q], 1);
+    }
+    for (int i = 0; i < kItemSlots; ++i) {
+      ptx::mbar_init(&bars->item_full[i], 1);
+      ptx::mbar_init(&bars->item_empty[i], kItemConsumers);
     }
     bars->abort = 0;
     ptx::fence_mbar_init();
@@ -520,9 +546,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t kv_tiles = 0;              // key tiles issued so far (ring position)
       uint32_t q_loads[2] = {0u, 0u};     // loads of each Q slot so far
       bool ok = true;
-      for (int rnd = 0; ok; ++rnd) {
-        const int w = item_of_round(rnd);
-        if (w >= num_items) break;
+      for (uint32_t k = 0; ok; ++k) {
+        int w = k == 0 ? static_cast<int>(blockIdx.x)
+                       : static_cast<int>(gridDim.x) + atomicAdd(p.ticket, 1);
+        if (w >= num_items) w = -1;
+        // publish it once every consumer has read the slot's previous item
+        // (item_empty's next phase needs this publication)
+        const int slot = k % kItemSlots;
+        if (k >= kItemSlots &&
+            !wait_bar(&bars->item_empty[slot], ((k / kItemSlots) - 1) & 1, abort_flag, tmo))
+          break;
+        *reinterpret_cast<volatile int*>(&bars->item_ring[slot]) = w;
+        ptx::mbar_arrive(&bars->item_full[slot]);
+        if (w < 0) break;
         WorkItem it;
         if (!load_item(p, w, it)) continue;
         // Q tile q's slot is refilled once the previous item's last S of it
@@ -605,9 +641,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t n_p = 0;       // P_q.V issued so far
       uint32_t n_items = 0;   // items that had a Q tile q
       bool ok = true;
-      for (int rnd = 0; ok; ++rnd) {
-        const int w = item_of_round(rnd);
-        if (w >= num_items) break;
+      for (uint32_t k = 0; ok; ++k) {
+        const int w = next_item(bars, k, abort_flag, tmo, false);
+        if (w == kItemAbort) {
+          ok = false;
+          break;
+        }
+        if (w < 0) break;
         WorkItem it;
         if (!load_item(p, w, it)) continue;
         const bool mine = q < it.nq;
@@ -703,9 +743,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t n_items = 0;  // items that had a Q tile q
     bool ok = true;
     uint32_t r[64];
-    for (int rnd = 0; ok; ++rnd) {
-      const int w = item_of_round(rnd);
-      if (w >= num_items) break;
+    for (uint32_t k = 0; ok; ++k) {
+      const int w = next_item(bars, k, abort_flag, tmo, true);
+      if (w == kItemAbort) {
+        ok = false;
+        break;
+      }
+      if (w < 0) break;
       WorkItem it;
       if (!load_item(p, w, it)) continue;
       if (q >= it.nq) continue;
@@ -841,7 +885,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ok = false;
         break;
       }
-      if (tr == 0 && q == 0 && rnd == 0) CTA_TRACE(3, gtimer());
+      if (tr == 0 && q == 0 && k == 0) CTA_TRACE(3, gtimer());
       ptx::tc_fence_after();
       const float inv_l = 1.0f / l;
       const bool valid = my_row < L;
