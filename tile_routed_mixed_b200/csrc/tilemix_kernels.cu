@@ -496,6 +496,148 @@ __device__ __forceinline__ bool load_item(const PrefillParams& p, int w, WorkIte
   return true;
 }
 
+// What one softmax thread needs about its row and Q tile for the key-tile
+// loop, and the row's running state.
+struct SoftmaxCtx {
+  const PrefillParams* p;
+  Barriers* bars;
+  volatile int* abort_flag;
+  unsigned long long tmo;
+  unsigned long long* trace_buf;  // profiling builds only
+  uint32_t ts, to, tp0;           // TMEM addresses of this lane's S, O and P buffer 0
+  int q, tr, L, row0, my_row, h, t0, ntq;
+  float q_sc;
+  const float* ks;                // K block scales of the sequence and KV head
+};
+struct RowState {
+  float m;          // running max, log2 units
+  float l;          // normaliser: sum of the fp16-rounded P actually used in P.V
+  float k_sc_next;  // K scale of the next key tile (loaded one tile ahead)
+  uint32_t n_s;     // S_q read so far
+  uint32_t n_p;     // P_q stored so far
+};
+
+// One key tile of the shared online softmax for this thread's row: S from
+// TMEM, the routed score domain, legality, max / normaliser update, lazy
+// rescale of O, P (fp16) to TMEM.  kCold adds what only the diagonal and
+// sequence-tail tiles (legality mask) and debug runs (INT32 dump) need; the
+// lean kMasked = false copy runs every other tile, so the hot loop carries
+// no code for them.  False if a wait gave up.
+template <int D, bool kCold>
+__device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st, int i, bool is_int,
+                                             uint32_t (&r)[64]) {
+#ifdef TILEMIX_TRACE
+  unsigned long long* const trace_buf = cx.trace_buf;
+#endif
+  const int q = cx.q, tr = cx.tr;
+  const int sb = st.n_p & 1;
+  const float k_sc = st.k_sc_next;
+  if (i + 1 < cx.ntq) st.k_sc_next = __ldg(cx.ks + i + 1);
+  // s_full's next phase needs s_free from this read
+  if (!wait_bar_warp(&cx.bars->s_full[q], st.n_s & 1, cx.abort_flag, cx.tmo)) return false;
+  ptx::tc_fence_after();
+  if (tr == 0) TRACE(0, q, i);
+  ptx::tmem_ld32(cx.ts, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  ptx::tmem_ld32(cx.ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  ptx::tmem_ld_wait();
+  // S is in registers: the MMA warp may compute the next S now
+  ptx::tc_fence_before();
+  ptx::mbar_arrive(&cx.bars->s_free[q]);
+  ++st.n_s;
+  if (tr == 0) TRACE(11, q, i);
+  const int key0 = i * BN;
+  if (kCold && is_int && cx.p->dbg && cx.my_row < cx.L) {
+    int32_t* drow = cx.p->dbg +
+                    (static_cast<size_t>(cx.h) * cx.p->total_tokens + cx.t0 + cx.my_row) * cx.p->dbg_cols;
+    for (int j = 0; j < 64; ++j)
+      if (key0 + j < cx.L) drow[key0 + j] = static_cast<int32_t>(r[j]);
+  }
+  // scores in the float domain, before the log2(e)-scaled softmax:
+  // FP16 tile: raw fp32 dot; INT8 tile: exact float of the INT32 dot.
+  if (is_int) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j) r[j] = __float_as_uint(__int2float_rn(static_cast<int>(r[j])));
+  }
+  const float c = is_int ? cx.q_sc * k_sc * cx.p->scale_log2 : cx.p->scale_log2;
+  const bool masked =
+      kCold && (key0 + BN > cx.L || (cx.p->causal && key0 + BN - 1 > cx.row0));
+  const int lim = cx.p->causal ? min(cx.L, cx.my_row + 1) : cx.L;  // legal keys < lim
+  if (masked) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j)
+      if (key0 + j >= lim) r[j] = __float_as_uint(-INFINITY);
+  }
+  // row max of the tile: eight independent chains, then a short tree
+  float g8[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const float* x = reinterpret_cast<const float*>(&r[8 * u]);
+    g8[u] = fmaxf(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), x[6]), x[7]);
+  }
+  const float mx = fmaxf(max3(g8[0], g8[1], g8[2]), max3(max3(g8[3], g8[4], g8[5]), g8[6], g8[7]));
+  // c >= 0; c == 0 only for an all-zero quantisation block (scores 0)
+  const float m_tile = mx == -INFINITY ? -INFINITY : mx * c;
+  if (tr == 0) TRACE(12, q, i);
+  const float m_new = fmaxf(st.m, m_tile);
+  const bool resc = m_new - st.m > kRescaleThreshold;
+  const float m_use = resc ? m_new : st.m;
+  const float alpha = resc ? ptx::ex2(st.m - m_new) : 1.0f;
+  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+  // P = 2^(score * c - m), packed in place: pair k lands in r[k]
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float x0 = fmaf(__uint_as_float(r[2 * k]), c, -m_use);
+    const float x1 = fmaf(__uint_as_float(r[2 * k + 1]), c, -m_use);
+    r[k] = pack_f16x2(ptx::ex2(x0), ptx::ex2(x1));
+    add_f16x2_to_f32(ls[k & 3], r[k]);
+  }
+  if (masked && c == 0.f) {
+    // an all-zero block (c == 0) turns -inf scores into NaN: clear them (for
+    // c > 0 the masked keys already gave 2^-inf = 0)
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const uint32_t keep = (key0 + 2 * k < lim ? 0x0000ffffu : 0u) |
+                            (key0 + 2 * k + 1 < lim ? 0xffff0000u : 0u);
+      r[k] &= keep;
+    }
+    ls[0] = ls[1] = ls[2] = ls[3] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) add_f16x2_to_f32(ls[k & 3], r[k]);
+  }
+  st.l = st.l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+  st.m = m_use;
+  if (tr == 0) TRACE(15, q, i);
+  if (i > 0 && __any_sync(0xffffffffu, resc)) {
+    // O holds P.V of tiles < i: rescale this warp's rows once P(i-1).V has
+    // landed (rows without a max move multiply by 1).  The P.V of the previous
+    // tile is the (n_p - 1)-th; the next phase of its pv_done barrier needs
+    // p_full from this tile.
+    if (!wait_bar_warp(&cx.bars->pv_done[q][(st.n_p - 1) & 1], ((st.n_p - 1) >> 1) & 1,
+                       cx.abort_flag, cx.tmo))
+      return false;
+    ptx::tc_fence_after();
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      ptx::tmem_ld32(cx.to + cc * 32, o);
+      ptx::tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+      ptx::tmem_st32(cx.to + cc * 32, o);
+    }
+  }
+  // P buffer sb held the P stored two tiles ago.  Its P.V was issued before
+  // this tile's S by the same thread, and the commit that signalled S covers
+  // every MMA issued before it: no wait needed.
+  ptx::tmem_st32(cx.tp0 + 32 * sb, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
+  ptx::tmem_st_wait();
+  ptx::tc_fence_before();
+  ptx::mbar_arrive(&cx.bars->p_full[q][sb]);
+  ++st.n_p;
+  if (tr == 0) TRACE(1, q, i);
+  return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ PrefillParams p) {
@@ -785,125 +927,57 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const float q_sc = __ldg(p.q_scale + static_cast<size_t>(h) * p.total_qtiles + it.cq + it.qt0 + q);
       const float* ks = p.k_scale + static_cast<size_t>(kv) * p.total_ktiles + it.ck;
       (void)s;
-      float m = -INFINITY;  // running max, log2 units
-      float l = 0.f;        // normaliser: sum of the fp16-rounded P actually used in P.V
-      float k_sc_next = __ldg(ks);
+      SoftmaxCtx cx;
+      cx.p = &p;
+      cx.bars = bars;
+      cx.abort_flag = abort_flag;
+      cx.tmo = tmo;
+#ifdef TILEMIX_TRACE
+      cx.trace_buf = trace_buf;
+#else
+      cx.trace_buf = nullptr;
+#endif
+      cx.ts = tmem + lane_base + S::col_s(q);
+      cx.to = tmem + lane_base + S::col_o(q);
+      cx.tp0 = tmem + lane_base + S::col_p(q, 0);
+      cx.q = q;
+      cx.tr = tr;
+      cx.L = L;
+      cx.row0 = row0;
+      cx.my_row = my_row;
+      cx.h = h;
+      cx.t0 = t0;
+      cx.ntq = ntq;
+      cx.q_sc = q_sc;
+      cx.ks = ks;
+      RowState st;
+      st.m = -INFINITY;
+      st.l = 0.f;
+      st.k_sc_next = __ldg(ks);
+      st.n_s = n_s;
+      st.n_p = n_p;
+      // Key tiles before the first one that needs the legality mask (the
+      // diagonal tiles of a causal row, a sequence's ragged last tile) run the
+      // lean body; the rest, and every tile of a debug run, the full one.
+      int i_hot = ntq;
+      if (p.causal) i_hot = min(i_hot, row0 / BN);
+      if (L % BN) i_hot = min(i_hot, L / BN);
+      if (p.dbg) i_hot = 0;
       GroupCursor gc;
-      for (int i = 0; i < ntq; ++i, gc.next(gs)) {
-        const int sb = n_p & 1;
-        const bool is_int = gc.int8(word);
-        const float k_sc = k_sc_next;
-        if (i + 1 < ntq) k_sc_next = __ldg(ks + i + 1);
-        // s_full's next phase needs s_free from this read
-        if (!wait_bar_warp(&bars->s_full[q], n_s & 1, abort_flag, tmo)) {
+      int i = 0;
+      for (; i < i_hot; ++i, gc.next(gs))
+        if (!softmax_tile<D, false>(cx, st, i, gc.int8(word), r)) {
           ok = false;
           break;
         }
-        ptx::tc_fence_after();
-        if (tr == 0) TRACE(0, q, i);
-        const uint32_t ts = tmem + lane_base + S::col_s(q);
-        ptx::tmem_ld32(ts, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        ptx::tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        ptx::tmem_ld_wait();
-        // S is in registers: the MMA warp may compute the next S now
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->s_free[q]);
-        ++n_s;
-        if (tr == 0) TRACE(11, q, i);
-        if (is_int && p.dbg && my_row < L) {
-          int32_t* drow =
-              p.dbg + (static_cast<size_t>(h) * p.total_tokens + t0 + my_row) * p.dbg_cols;
-          for (int j = 0; j < 64; ++j)
-            if (i * BN + j < L) drow[i * BN + j] = static_cast<int32_t>(r[j]);
+      for (; ok && i < ntq; ++i, gc.next(gs))
+        if (!softmax_tile<D, true>(cx, st, i, gc.int8(word), r)) {
+          ok = false;
+          break;
         }
-        // scores in the float domain, before the log2(e)-scaled softmax:
-        // FP16 tile: raw fp32 dot; INT8 tile: exact float of the INT32 dot.
-        if (is_int) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) r[j] = __float_as_uint(__int2float_rn(static_cast<int>(r[j])));
-        }
-        const float c = is_int ? q_sc * k_sc * p.scale_log2 : p.scale_log2;
-        const int key0 = i * BN;
-        const bool masked = key0 + BN > L || (p.causal && key0 + BN - 1 > row0);
-        const int lim = p.causal ? min(L, my_row + 1) : L;  // legal keys < lim
-        if (masked) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (key0 + j >= lim) r[j] = __float_as_uint(-INFINITY);
-        }
-        // row max of the tile: eight independent chains, then a short tree
-        float g8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float* x = reinterpret_cast<const float*>(&r[8 * u]);
-          g8[u] = fmaxf(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), x[6]), x[7]);
-        }
-        const float mx = fmaxf(max3(g8[0], g8[1], g8[2]), max3(max3(g8[3], g8[4], g8[5]), g8[6], g8[7]));
-        // c >= 0; c == 0 only for an all-zero quantisation block (scores 0)
-        const float m_tile = mx == -INFINITY ? -INFINITY : mx * c;
-        if (tr == 0) TRACE(12, q, i);
-        const float m_new = fmaxf(m, m_tile);
-        const bool resc = m_new - m > kRescaleThreshold;
-        const float m_use = resc ? m_new : m;
-        const float alpha = resc ? ptx::ex2(m - m_new) : 1.0f;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-        // P = 2^(score * c - m), packed in place: pair k lands in r[k]
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float x0 = fmaf(__uint_as_float(r[2 * k]), c, -m_use);
-          const float x1 = fmaf(__uint_as_float(r[2 * k + 1]), c, -m_use);
-          r[k] = pack_f16x2(ptx::ex2(x0), ptx::ex2(x1));
-          add_f16x2_to_f32(ls[k & 3], r[k]);
-        }
-        if (masked) {
-          // an all-zero block (c == 0) turns -inf scores into NaN: clear them
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const uint32_t keep = (key0 + 2 * k < lim ? 0x0000ffffu : 0u) |
-                                  (key0 + 2 * k + 1 < lim ? 0xffff0000u : 0u);
-            r[k] &= keep;
-          }
-          if (c == 0.f) {
-            ls[0] = ls[1] = ls[2] = ls[3] = 0.f;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) add_f16x2_to_f32(ls[k & 3], r[k]);
-          }
-        }
-        l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-        m = m_use;
-        if (tr == 0) TRACE(15, q, i);
-        if (i > 0 && __any_sync(0xffffffffu, resc)) {
-          // O holds P.V of tiles < i: rescale this warp's rows once P(i-1).V
-          // has landed (rows without a max move multiply by 1)
-          // (the P.V of the previous tile is the (n_p - 1)-th; the next phase
-          // of its pv_done barrier needs p_full from this tile)
-          if (!wait_bar_warp(&bars->pv_done[q][(n_p - 1) & 1], ((n_p - 1) >> 1) & 1, abort_flag, tmo)) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            const uint32_t to = tmem + lane_base + S::col_o(q) + cc * 32;
-            ptx::tmem_ld32(to, o);
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            ptx::tmem_st32(to, o);
-          }
-        }
-        // P buffer sb held the P stored two tiles ago.  Its P.V was issued
-        // before this tile's S by the same thread, and the commit that
-        // signalled S covers every MMA issued before it: no wait needed.
-        ptx::tmem_st32(tmem + lane_base + S::col_p(q, sb),
-                       *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->p_full[q][sb]);
-        ++n_p;
-        if (tr == 0) TRACE(1, q, i);
-      }
+      n_s = st.n_s;
+      n_p = st.n_p;
+      const float m = st.m, l = st.l;
       // o_final's next phase needs o_free from this epilogue
       if (!ok || !wait_bar_warp(&bars->o_final[q], n_items & 1, abort_flag, tmo)) {
         ok = false;
