@@ -519,11 +519,11 @@ struct RowState {
 
 // One key tile of the shared online softmax for this thread's row: S from
 // TMEM, the routed score domain, legality, max / normaliser update, lazy
-// rescale of O, P (fp16) to TMEM.  kCold adds what only the diagonal and
-// sequence-tail tiles (legality mask) and debug runs (INT32 dump) need; the
-// lean kMasked = false copy runs every other tile, so the hot loop carries
-// no code for them.  False if a wait gave up.
-template <int D, bool kCold>
+// rescale of O, P (fp16) to TMEM.  kMask adds the legality mask that only the
+// diagonal and sequence-tail tiles need, kDebug the INT32 score dump of debug
+// runs; the lean copy runs every other tile, so the hot loop carries no code
+// for them.  False if a wait gave up.
+template <int D, bool kMask, bool kDebug>
 __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st, int i, bool is_int,
                                              uint32_t (&r)[64]) {
 #ifdef TILEMIX_TRACE
@@ -546,7 +546,7 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st,
   ++st.n_s;
   if (tr == 0) TRACE(11, q, i);
   const int key0 = i * BN;
-  if (kCold && is_int && cx.p->dbg && cx.my_row < cx.L) {
+  if (kDebug && is_int && cx.p->dbg && cx.my_row < cx.L) {
     int32_t* drow = cx.p->dbg +
                     (static_cast<size_t>(cx.h) * cx.p->total_tokens + cx.t0 + cx.my_row) * cx.p->dbg_cols;
     for (int j = 0; j < 64; ++j)
@@ -560,7 +560,7 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st,
   }
   const float c = is_int ? cx.q_sc * k_sc * cx.p->scale_log2 : cx.p->scale_log2;
   const bool masked =
-      kCold && (key0 + BN > cx.L || (cx.p->causal && key0 + BN - 1 > cx.row0));
+      kMask && (key0 + BN > cx.L || (cx.p->causal && key0 + BN - 1 > cx.row0));
   const int lim = cx.p->causal ? min(cx.L, cx.my_row + 1) : cx.L;  // legal keys < lim
   if (masked) {
 #pragma unroll
@@ -958,20 +958,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       st.n_p = n_p;
       // Key tiles before the first one that needs the legality mask (the
       // diagonal tiles of a causal row, a sequence's ragged last tile) run the
-      // lean body; the rest, and every tile of a debug run, the full one.
+      // lean body, the rest the masked one; a debug run takes the body with
+      // the INT32 dump for every tile.
       int i_hot = ntq;
       if (p.causal) i_hot = min(i_hot, row0 / BN);
       if (L % BN) i_hot = min(i_hot, L / BN);
-      if (p.dbg) i_hot = 0;
       GroupCursor gc;
       int i = 0;
-      for (; i < i_hot; ++i, gc.next(gs))
-        if (!softmax_tile<D, false>(cx, st, i, gc.int8(word), r)) {
+      if (p.dbg) {
+        for (; i < ntq; ++i, gc.next(gs))
+          if (!softmax_tile<D, true, true>(cx, st, i, gc.int8(word), r)) {
+            ok = false;
+            break;
+          }
+      }
+      for (; ok && i < i_hot; ++i, gc.next(gs))
+        if (!softmax_tile<D, false, false>(cx, st, i, gc.int8(word), r)) {
           ok = false;
           break;
         }
       for (; ok && i < ntq; ++i, gc.next(gs))
-        if (!softmax_tile<D, true>(cx, st, i, gc.int8(word), r)) {
+        if (!softmax_tile<D, true, false>(cx, st, i, gc.int8(word), r)) {
           ok = false;
           break;
         }
