@@ -451,13 +451,20 @@ struct WorkItem {
   uint64_t w0, w1;
 };
 
-// Decodes item w (heaviest query-tile pairs first, heads innermost).  False
-// if the sequence has no such pair, or if its routing would need a group
-// index above 63 (reported in the status word).
+// Decodes item w.  Items are ordered by (sequence, KV head), then query-tile
+// pair heaviest first, then the KV head's query heads, so that the CTAs
+// working at any one time share the K/V of a few heads and those stay in L2,
+// while each group's lightest items come last.  (With a custom head map the
+// order is only a heuristic; every (s, h, pair) is still visited once.)
+// False if the sequence has no such pair, or if its routing would need a
+// group index above 63 (reported in the status word).
 __device__ __forceinline__ bool load_item(const PrefillParams& p, int w, WorkItem& it) {
-  const int h = w % p.hq;
-  const int s = (w / p.hq) % p.nseq;
-  const int pair = p.max_qpairs - 1 - w / (p.hq * p.nseq);
+  const int per_kv = p.max_qpairs * p.group;
+  const int kvg = w / per_kv;  // (s, kv) index, sequence-major
+  const int rem = w - kvg * per_kv;
+  const int pair = p.max_qpairs - 1 - rem / p.group;
+  const int h = (kvg % p.hk) * p.group + rem % p.group;
+  const int s = kvg / p.hk;
   // independent loads first, so that they overlap
   const int t0 = __ldg(p.cu_seqlens + s);
   const int t1 = __ldg(p.cu_seqlens + s + 1);
