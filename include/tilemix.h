@@ -209,6 +209,67 @@ int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
 #define TILEMIX_NOALLOC_SCRATCH_BYTES (64u << 20)
 int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Decode with the INT8 K cache: one new query token per sequence.
+ *
+ * The step after prefill named by the pages ("TileMix: Tile-Centric Mixed-
+ * Precision Attention for LLM Inference Acceleration", agihunt.info summary;
+ * "Precision Has a Map: TileMix Routes INT8 Inside Dense Attention",
+ * cognaptus.com, last section): the INT8 K codes and 64-key block scales of
+ * the quantisation pre-pass serve as the K cache, and a new token's query
+ * reads the routing word of its query-tile row.  The pages give no decode
+ * algorithm; this library reads it as the prefill method applied to one row:
+ *   - sequence s holds seq_len[s] >= 1 cached tokens in cache rows
+ *     [seq_start[s], seq_start[s] + seq_len[s]); the new token is the last
+ *     one, at position t = seq_len[s] - 1, its K and V already written, and it
+ *     attends to positions 0..t (causal);
+ *   - key tile kt (keys 64 kt .. 64 kt + 63) uses the INT8 score path iff bit
+ *     (kt / g[s]) of masks[(qtile_start[s] + t / 128) * hk + kv] is set;
+ *   - the query is quantised as a block of its own (one row: earlier queries
+ *     are not kept), symmetric absmax / 127 with the prefill rounding rules;
+ *   - this call re-quantises the K block holding the new key (rows
+ *     64 * (t / 64) .. t of the sequence) over its valid rows and writes its
+ *     codes and scale into k_i8 / k_scale; every other block must already be
+ *     current there (as tilemix_quantize_qk leaves them);
+ *   - softmax state in fp32, P rounded to fp16 before P.V, O rounded once to
+ *     fp16, as in the prefill path.
+ * Three launches on `stream`: quantisation (last K blocks, query rows), split
+ * attention over key ranges, merge.  Bad routing factors are reported by
+ * tilemix_get_error() as for prefill. */
+typedef struct tilemix_decode_args {
+  const void* q;              /* device fp16 [nseq][hq][d]: the new tokens' queries, 16-B aligned */
+  const void* k;              /* device fp16 [cache_rows][hk][d], 16-B aligned */
+  const void* v;              /* device fp16 [cache_rows][hk][d], 16-B aligned */
+  int8_t* k_i8;               /* device int8 [cache_rows][hk][d], 16-B aligned: INT8 K cache */
+  float* k_scale;             /* device fp32 [hk][total_ktiles]: K block scales */
+  void* o;                    /* device fp16 [nseq][hq][d] */
+  const int32_t* seq_start;   /* device [nseq]: first cache row of each sequence */
+  const int32_t* seq_len;     /* device [nseq]: tokens in the cache incl. the new one, >= 1 */
+  const int32_t* ktile_start; /* device [nseq]: k_scale column of each sequence's first K block */
+  const int32_t* qtile_start; /* device [nseq]: masks row of each sequence's first query tile */
+  const uint64_t* masks;      /* device [total_qtiles][hk] routing words */
+  const int32_t* g;           /* device [nseq] routing-group factors */
+  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk) */
+  int nseq;                   /* >= 0 (0: nothing to do) */
+  int max_seqlen;             /* >= every seq_len[s] (sizes the split of the key range) */
+  int total_ktiles;           /* columns of k_scale */
+  int hq, hk, d;              /* d in {64, 128}; hq % hk == 0; at most 16 query heads per KV head */
+  float softmax_scale;        /* 0 => 1 / sqrt(d) */
+  void* workspace;            /* device, >= tilemix_decode_workspace_size(), 256-aligned */
+  size_t workspace_bytes;
+} tilemix_decode_args;
+
+/* Bytes of device workspace tilemix_decode_fwd needs (query codes and the
+ * split attention's partial states).  INVALID_ARG / UNSUPPORTED as for
+ * tilemix_decode_fwd. */
+int tilemix_decode_workspace_size(const tilemix_decode_args* args, size_t* bytes);
+
+/* Decode step as described above.  INVALID_ARG on a NULL required pointer, a
+ * misaligned tensor, nseq < 0, max_seqlen < 1 or hq % hk != 0; UNSUPPORTED for
+ * d not in {64, 128} or more than 16 query heads per KV head; WORKSPACE if the
+ * workspace is missing, misaligned or too small; CUDA if a launch fails. */
+int tilemix_decode_fwd(const tilemix_decode_args* args, void* stream);
+
 /* Self test of the failure path: enqueues one warp that waits on a device
  * barrier nothing ever signals, with the same bounded wait the attention
  * kernel uses, limited to timeout_ms (1..10000).  The wait gives up, latches

@@ -141,3 +141,38 @@ def test_prefill_argument_checks_are_synchronous():
                                  None, None, None) == tm.OK
     assert L.tilemix_quantize_qk(None, None, None, None, None, 1, 10, 1, 1, 1, 1, 80, None,
                                  None, None, None, None) == tm.ERR_UNSUPPORTED
+
+
+def _fake_decode(**over):
+    a = tm.DecodeArgs()
+    for f in ("q", "k", "v", "k_i8", "k_scale", "o", "seq_start", "seq_len", "ktile_start",
+              "qtile_start", "masks", "g"):
+        setattr(a, f, 4096)
+    a.nseq, a.max_seqlen, a.total_ktiles = 2, 300, 10
+    a.hq, a.hk, a.d = 6, 2, 128
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_decode_argument_checks_are_synchronous():
+    L = tm.lib()
+    n = ctypes.c_size_t(0)
+    assert L.tilemix_decode_workspace_size(ctypes.byref(_fake_decode()), ctypes.byref(n)) == tm.OK
+    assert n.value > 0
+    cases = [
+        (dict(d=80), tm.ERR_UNSUPPORTED),
+        (dict(hq=6, hk=4), tm.ERR_INVALID_ARG),
+        (dict(hq=34, hk=2), tm.ERR_UNSUPPORTED),        # 17 query heads per KV head
+        (dict(max_seqlen=0), tm.ERR_INVALID_ARG),
+        (dict(nseq=-1), tm.ERR_INVALID_ARG),
+        (dict(k_i8=None), tm.ERR_INVALID_ARG),
+        (dict(q=4097), tm.ERR_INVALID_ARG),             # misaligned
+        (dict(softmax_scale=-1.0), tm.ERR_INVALID_ARG),
+        (dict(workspace=None), tm.ERR_WORKSPACE),
+        (dict(workspace=4096 + 128, workspace_bytes=1 << 30), tm.ERR_WORKSPACE),  # misaligned
+    ]
+    for over, want in cases:
+        assert L.tilemix_decode_fwd(ctypes.byref(_fake_decode(**over)), None) == want, over
+    # nothing to do: OK without touching any pointer
+    assert L.tilemix_decode_fwd(ctypes.byref(_fake_decode(nseq=0, q=None)), None) == tm.OK

@@ -1,0 +1,111 @@
+"""GPU parity of the decode step with the INT8 K cache (tilemix_decode_fwd)
+against the oracle: the re-quantised last K blocks bit for bit, O within
+max-abs 2e-3 / mean-abs 2e-4."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import gpu_cases as gc
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    gc.set_test_timeout()
+
+
+def _run(lengths, hq, hk, d, masks_fn, g, seed, slack=37, kv_map=None):
+    import tile_routed_mixed_b200 as tm
+    rng = np.random.default_rng(seed)
+    nseq = len(lengths)
+    starts, ktiles, a, kt = [], [], 0, 0
+    for L in lengths:
+        starts.append(a)
+        ktiles.append(kt)
+        a += L + slack                       # cache capacity beyond the current length
+        kt += (L + slack + 63) // 64
+    rows, total_kt = a, kt
+    k = synth.fp16_normal(seed, 2, (rows, hk, d))
+    v = synth.fp16_normal(seed, 3, (rows, hk, d))
+    q = synth.fp16_normal(seed, 1, (nseq, hq, d))
+    qt = np.zeros(nseq + 1, dtype=np.int64)
+    qt[1:] = np.cumsum([(L + 127) // 128 for L in lengths])
+    masks = masks_fn(int(qt[-1]))
+    # INT8 K cache as the previous steps left it: every block current except
+    # the one holding the new key, which is stale
+    k8 = np.zeros((rows, hk, d), dtype=np.int8)
+    ks = np.zeros((hk, total_kt), dtype=np.float32)
+    want_k8, want_ks = k8.copy(), ks.copy()
+    for s, L in enumerate(lengths):
+        c, sc = oracle.quantize_k(np.ascontiguousarray(k[starts[s]:starts[s] + L]), [L])
+        want_k8[starts[s]:starts[s] + L] = c
+        want_ks[:, ktiles[s]:ktiles[s] + sc.shape[1]] = sc
+        k8[starts[s]:starts[s] + L] = c
+        ks[:, ktiles[s]:ktiles[s] + sc.shape[1]] = sc
+        b = (L - 1) // 64
+        k8[starts[s] + 64 * b:starts[s] + L] = 99
+        ks[:, ktiles[s] + b] = -1.0
+    dev = "cuda"
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+    dec = tm.TileMixDecode(starts, lengths, ktiles, qt[:-1], hq, hk, d, masks, g, total_kt,
+                           kv_head_of_q=kv_map, device=dev)
+    qd, kd, vd, k8d, ksd = t(q), t(k), t(v), t(k8), t(ks)
+    o = dec(qd, kd, vd, k8d, ksd)
+    torch.cuda.synchronize()
+    assert tm.tilemix_get_error() == tm.OK
+    got_k8, got_ks = k8d.cpu().numpy(), ksd.cpu().numpy()
+    for s, L in enumerate(lengths):
+        assert np.array_equal(got_k8[starts[s]:starts[s] + L], want_k8[starts[s]:starts[s] + L])
+    assert np.array_equal(got_ks.view(np.uint32), want_ks.view(np.uint32))
+    want, _ = oracle.decode_rows(q, k, v, starts, lengths, masks, qt[:-1], g, kv_map=kv_map)
+    got = o.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    mx, mn = gc.errors(got.reshape(-1, d), want.reshape(-1, d))
+    assert mx <= gc.MAX_ABS and mn <= gc.MEAN_ABS, (mx, mn)
+    return mx, mn
+
+
+def _template(name, percent, lengths, hk, g):
+    def f(nqt):
+        m, _, _ = oracle.build_routing(name, percent, 0, lengths, hk, g, True)
+        assert m.shape == (nqt, hk)
+        return m
+    return f
+
+
+@pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 200, 1000], [4096] * 8])
+def test_decode_sptrans_ragged(lengths):
+    g = np.ones(len(lengths), dtype=np.int32)
+    _run(lengths, 24 if len(lengths) == 8 else 6, 8 if len(lengths) == 8 else 2, 128,
+         _template("sptrans", 75, lengths, 8 if len(lengths) == 8 else 2, g), g, seed=5)
+
+
+def test_decode_d64_gqa4_bigbird_g2():
+    lengths = [129, 640, 33]
+    g = np.full(len(lengths), 2, dtype=np.int32)
+    _run(lengths, 4, 1, 64, _template("bigbird", 50, lengths, 1, g), g, seed=6)
+
+
+@pytest.mark.parametrize("word", [0, 2 ** 64 - 1])
+def test_decode_all_fp16_and_all_int8(word):
+    lengths = [77, 300]
+    g = np.ones(2, dtype=np.int32)
+    _run(lengths, 8, 2, 128, lambda n: np.full((n, 2), np.uint64(word), dtype=np.uint64), g, seed=7)
+
+
+def test_decode_custom_head_map():
+    lengths = [150, 90]
+    g = np.ones(2, dtype=np.int32)
+    kv_map = np.array([1, 0, 1, 0, 0, 1], dtype=np.int32)
+    _run(lengths, 6, 2, 128, _template("row_random", 50, lengths, 2, g), g, seed=8, kv_map=kv_map)
+
+
+def test_decode_long_context():
+    lengths = [16384, 5000]
+    g = np.array([oracle.auto_g(L) for L in lengths], dtype=np.int32)
+    _run(lengths, 8, 2, 128, _template("row_random", 25, lengths, 2, g), g, seed=9)

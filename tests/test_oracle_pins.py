@@ -419,3 +419,96 @@ def test_deviation_grows_with_coverage():
         mads.append(np.abs(O - base).mean())
     assert mads[0] == 0.0
     assert all(b >= a for a, b in zip(mads, mads[1:]))
+
+
+# ------------------------------------------------------------------ decode ---
+# The decode step (one new query row per sequence attending to its cache) is
+# the prefill row oracle composed with a single-row query block; these pins
+# check the composition against whole-matrix brute force.
+
+def _decode_case(lengths, hq, hk, d, seed, slack=5):
+    rng = np.random.default_rng(seed)
+    starts, a = [], 0
+    for L in lengths:
+        starts.append(a)
+        a += L + slack                      # caches with capacity slack between sequences
+    rows = a
+    k = rng.standard_normal((rows, hk, d)).astype(np.float16)
+    v = rng.standard_normal((rows, hk, d)).astype(np.float16)
+    q = rng.standard_normal((len(lengths), hq, d)).astype(np.float16)
+    qt = [0]
+    for L in lengths:
+        qt.append(qt[-1] + (L + 127) // 128)
+    return q, k, v, np.array(starts), np.array(lengths), np.array(qt[:-1]), qt[-1]
+
+
+@pytest.mark.parametrize("lengths,hq,hk,d", [([1, 64, 65, 200], 4, 2, 64), ([130, 7], 3, 1, 128)])
+def test_decode_all_fp16_equals_softmax_of_the_new_row(lengths, hq, hk, d):
+    q, k, v, st, ln, qts, nqt = _decode_case(lengths, hq, hk, d, 1)
+    masks = np.zeros((nqt, hk), dtype=np.uint64)
+    o, lse = oracle.decode_rows(q, k, v, st, ln, masks, qts, np.ones(len(lengths), np.int32))
+    for s, L in enumerate(lengths):
+        qs = np.zeros((L, hq, d), dtype=np.float16)
+        qs[L - 1] = q[s]
+        want, wl = bf.naive_attention(qs, k[st[s]:st[s] + L], v[st[s]:st[s] + L], [L], True)
+        assert np.abs(o[s] - want[L - 1]).max() < 1e-12
+        assert np.abs(lse[s] - wl[:, L - 1]).max() < 1e-12
+
+
+@pytest.mark.parametrize("lengths,hq,hk,d", [([1, 63, 64, 129], 2, 2, 64), ([300], 4, 2, 128)])
+def test_decode_all_int8_equals_integer_bruteforce(lengths, hq, hk, d):
+    q, k, v, st, ln, qts, nqt = _decode_case(lengths, hq, hk, d, 2)
+    masks = np.full((nqt, hk), np.uint64(2 ** 64 - 1), dtype=np.uint64)
+    o, _ = oracle.decode_rows(q, k, v, st, ln, masks, qts, np.ones(len(lengths), np.int32))
+    scale = 1.0 / math.sqrt(d)
+    for s, L in enumerate(lengths):
+        K, V = k[st[s]:st[s] + L], v[st[s]:st[s] + L]
+        k8, ks = oracle.quantize_k(K, [L])              # pinned above
+        for h in range(hq):
+            kv = h // (hq // hk)
+            x = q[s, h].astype(np.float32)
+            a = np.float32(np.abs(x).max())
+            sq = np.float32(a / np.float32(127.0))
+            q8 = np.clip(np.rint(x / sq), -127, 127).astype(np.int64)
+            dots = k8[:, kv].astype(np.int64) @ q8       # exact integers, [L]
+            sk = ks[kv, np.arange(L) // 64].astype(np.float64)
+            S = dots.astype(np.float64) * float(sq) * sk * scale
+            P = np.exp(S - S.max())
+            want = (P @ V[:, kv].astype(np.float64)) / P.sum()
+            assert np.abs(o[s, h] - want).max() < 1e-12
+
+
+def test_decode_matches_prefill_row_when_the_query_tile_is_the_new_row():
+    # with an all-FP16 word the query quantisation plays no part: the decode of
+    # position t equals the prefill oracle's row t of the same sequence
+    L, hq, hk, d = 100, 2, 1, 64
+    q, k, v, st, ln, qts, nqt = _decode_case([L], hq, hk, d, 3, slack=0)
+    qs = np.zeros((L, hq, d), dtype=np.float16)
+    qs[L - 1] = q[0]
+    masks = np.zeros((nqt, hk), dtype=np.uint64)
+    o, _ = oracle.decode_rows(q, k, v, st, ln, masks, qts, np.ones(1, np.int32))
+    q8, qsc = oracle.quantize_q(qs, [L])
+    k8, ksc = oracle.quantize_k(k, [L])
+    want, _ = oracle.attention_rows(qs, k, v, q8, qsc, k8, ksc, masks, np.ones(1, np.int32), [L],
+                                    True, rows=np.array([(0, h, L - 1) for h in range(hq)]))
+    assert np.abs(o[0] - want).max() < 1e-12
+
+
+def test_decode_reads_the_word_of_the_new_rows_query_tile():
+    # row 0 of the sequence's words says all INT8, row 1 (where t = 199 lives)
+    # all FP16: the result is the FP16 one
+    L, hq, hk, d = 200, 2, 1, 64
+    q, k, v, st, ln, qts, nqt = _decode_case([L], hq, hk, d, 4, slack=0)
+    masks = np.array([[2 ** 64 - 1], [0]], dtype=np.uint64)
+    o, _ = oracle.decode_rows(q, k, v, st, ln, masks, qts, np.ones(1, np.int32))
+    o16, _ = oracle.decode_rows(q, k, v, st, ln, np.zeros_like(masks), qts, np.ones(1, np.int32))
+    assert np.abs(o - o16).max() == 0.0
+
+
+def test_decode_query_rows_are_their_own_blocks():
+    x = np.zeros((2, 1, 64), dtype=np.float16)
+    x[0, 0, :3] = [127.0, -63.5, 0.5]       # a = 127 -> s = 1: rne(-63.5) = -64, rne(0.5) = 0
+    x[1, 0, 0] = 2.0                        # a second row with its own scale
+    c, s = oracle.quantize_rows(x)
+    assert list(c[0, 0, :3]) == [127, -64, 0] and s[0, 0] == np.float32(1.0)
+    assert c[1, 0, 0] == 127 and s[1, 0] == np.float32(np.float32(2.0) / np.float32(127.0))

@@ -52,6 +52,21 @@ class PrefillArgs(ctypes.Structure):
     ]
 
 
+class DecodeArgs(ctypes.Structure):
+    """Mirror of ``tilemix_decode_args``."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("k_i8", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("o", ctypes.c_void_p),
+        ("seq_start", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
+        ("ktile_start", ctypes.c_void_p), ("qtile_start", ctypes.c_void_p),
+        ("masks", ctypes.c_void_p), ("g", ctypes.c_void_p), ("kv_head_of_q", ctypes.c_void_p),
+        ("nseq", ctypes.c_int), ("max_seqlen", ctypes.c_int), ("total_ktiles", ctypes.c_int),
+        ("hq", ctypes.c_int), ("hk", ctypes.c_int), ("d", ctypes.c_int),
+        ("softmax_scale", ctypes.c_float),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 _lib = None
 
 
@@ -82,6 +97,11 @@ def lib():
         L.tilemix_prefill_fwd.argtypes = [ctypes.POINTER(PrefillArgs), P]
         L.tilemix_prefill_fwd_noalloc.restype = I
         L.tilemix_prefill_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), P]
+        L.tilemix_decode_workspace_size.restype = I
+        L.tilemix_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs),
+                                                    ctypes.POINTER(ctypes.c_size_t)]
+        L.tilemix_decode_fwd.restype = I
+        L.tilemix_decode_fwd.argtypes = [ctypes.POINTER(DecodeArgs), P]
         L.tilemix_selftest_wait_timeout.restype = I
         L.tilemix_selftest_wait_timeout.argtypes = [I, P]
         L.tilemix_get_error.restype = I
@@ -232,12 +252,26 @@ def tilemix_get_error(stream=None) -> int:
     return int(lib().tilemix_get_error(_stream_handle(stream)))
 
 
+def tilemix_decode_workspace_size(args: DecodeArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tilemix_decode_workspace_size(ctypes.byref(args), ctypes.byref(n)),
+           "tilemix_decode_workspace_size")
+    return int(n.value)
+
+
+def tilemix_decode_fwd(args: DecodeArgs, stream=None):
+    _check(lib().tilemix_decode_fwd(ctypes.byref(args), _stream_handle(stream)),
+           "tilemix_decode_fwd")
+
+
 from .prefill import TileMixPrefill  # noqa: E402  (convenience wrapper)
+from .decode import TileMixDecode  # noqa: E402  (convenience wrapper)
 
 __all__ = [
-    "BLOCK_M", "BLOCK_N", "MAX_GROUPS", "PrefillArgs", "TEMPLATES", "TileMixError",
-    "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
-    "tilemix_build_routing", "tilemix_get_error", "tilemix_prefill_fwd",
+    "BLOCK_M", "BLOCK_N", "DecodeArgs", "MAX_GROUPS", "PrefillArgs", "TEMPLATES", "TileMixError",
+    "TileMixDecode", "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
+    "tilemix_build_routing", "tilemix_decode_fwd", "tilemix_decode_workspace_size",
+    "tilemix_get_error", "tilemix_prefill_fwd",
     "tilemix_prefill_fwd_noalloc", "tilemix_quantize_qk", "tilemix_selftest_wait_timeout",
     "tilemix_status_string", "tilemix_tile_offsets", "tilemix_version",
     "tilemix_workspace_size",

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtilemix.so")
 SOURCES = ["tilemix_kernels.cu", "api.cpp", "routing.cpp"]
-HEADERS = ["tilemix_internal.h", "tilemix_ptx.cuh"]
+HEADERS = ["tilemix_internal.h", "tilemix_ptx.cuh", "tilemix_quant.cuh", "tilemix_decode.cuh"]
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",
     "-gencode", "arch=compute_100a,code=sm_100a",

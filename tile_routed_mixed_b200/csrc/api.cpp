@@ -271,6 +271,119 @@ TILEMIX_API int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, vo
   return tilemix_prefill_fwd(&a, stream);
 }
 
+namespace {
+
+struct DecodeLayout {
+  size_t q8, q_scale, part_m, part_l, part_acc, total;
+  int nsplit, tiles_per_split;
+};
+
+int check_decode(const tilemix_decode_args* a) {
+  if (!a) return TILEMIX_ERR_INVALID_ARG;
+  if (a->d != 64 && a->d != 128) return TILEMIX_ERR_UNSUPPORTED;
+  if (a->hq < 1 || a->hk < 1 || a->hq % a->hk != 0) return TILEMIX_ERR_INVALID_ARG;
+  if (a->kv_head_of_q == nullptr && a->hq / a->hk > 16) return TILEMIX_ERR_UNSUPPORTED;
+  if (a->nseq < 0 || a->max_seqlen < 1 || a->total_ktiles < 0) return TILEMIX_ERR_INVALID_ARG;
+  if (!(a->softmax_scale >= 0.f) || std::isinf(a->softmax_scale)) return TILEMIX_ERR_INVALID_ARG;
+  if (a->nseq == 0) return TILEMIX_OK;
+  if (!a->q || !a->k || !a->v || !a->k_i8 || !a->k_scale || !a->o || !a->seq_start ||
+      !a->seq_len || !a->ktile_start || !a->qtile_start || !a->masks || !a->g)
+    return TILEMIX_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->k_i8) ||
+      !aligned16(a->o))
+    return TILEMIX_ERR_INVALID_ARG;
+  return TILEMIX_OK;
+}
+
+int decode_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return 148;
+  return sms;
+}
+
+// The key range of every (sequence, KV head) is cut into nsplit pieces so that
+// about two CTAs per SM run the attention step.
+DecodeLayout decode_layout(const tilemix_decode_args* a) {
+  DecodeLayout w{};
+  const int max_tiles = (a->max_seqlen + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N;
+  const long long units = static_cast<long long>(a->nseq) * a->hk;
+  long long ns = units > 0 ? (2LL * decode_sms() + units - 1) / units : 1;
+  if (ns < 1) ns = 1;
+  if (ns > max_tiles) ns = max_tiles;
+  w.nsplit = static_cast<int>(ns);
+  w.tiles_per_split = (max_tiles + w.nsplit - 1) / w.nsplit;
+  const size_t rows = static_cast<size_t>(a->nseq) * a->hq;
+  size_t off = 0;
+  w.q8 = off;
+  off = round_up(off + rows * a->d, 256);
+  w.q_scale = off;
+  off = round_up(off + rows * sizeof(float), 256);
+  w.part_m = off;
+  off = round_up(off + rows * w.nsplit * sizeof(float), 256);
+  w.part_l = off;
+  off = round_up(off + rows * w.nsplit * sizeof(float), 256);
+  w.part_acc = off;
+  off = round_up(off + rows * w.nsplit * a->d * sizeof(float), 256);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+TILEMIX_API int tilemix_decode_workspace_size(const tilemix_decode_args* args, size_t* bytes) {
+  if (!args || !bytes) return TILEMIX_ERR_INVALID_ARG;
+  const int rc = check_decode(args);
+  if (rc != TILEMIX_OK) return rc;
+  *bytes = args->nseq == 0 ? 0 : decode_layout(args).total;
+  return TILEMIX_OK;
+}
+
+TILEMIX_API int tilemix_decode_fwd(const tilemix_decode_args* a, void* stream) {
+  int rc = check_decode(a);
+  if (rc != TILEMIX_OK) return rc;
+  if (a->nseq == 0) return TILEMIX_OK;
+  const DecodeLayout w = decode_layout(a);
+  if (!a->workspace || a->workspace_bytes < w.total ||
+      (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return TILEMIX_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  tilemix::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.k_i8 = a->k_i8;
+  p.k_scale = a->k_scale;
+  p.o = a->o;
+  p.seq_start = a->seq_start;
+  p.seq_len = a->seq_len;
+  p.ktile_start = a->ktile_start;
+  p.qtile_start = a->qtile_start;
+  p.masks = a->masks;
+  p.g = a->g;
+  p.kv_head_of_q = a->kv_head_of_q;
+  p.q8 = reinterpret_cast<int8_t*>(ws + w.q8);
+  p.q_scale = reinterpret_cast<float*>(ws + w.q_scale);
+  p.part_m = reinterpret_cast<float*>(ws + w.part_m);
+  p.part_l = reinterpret_cast<float*>(ws + w.part_l);
+  p.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
+  p.nseq = a->nseq;
+  p.hq = a->hq;
+  p.hk = a->hk;
+  p.d = a->d;
+  p.group = a->hq / a->hk;
+  p.total_ktiles = a->total_ktiles;
+  p.nsplit = w.nsplit;
+  p.tiles_per_split = w.tiles_per_split;
+  const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(a->d));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (tilemix::launch_decode(p, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  return TILEMIX_OK;
+}
+
 TILEMIX_API int tilemix_selftest_wait_timeout(int timeout_ms, void* stream) {
   if (timeout_ms < 1 || timeout_ms > 10000) return TILEMIX_ERR_INVALID_ARG;
   if (tilemix::launch_selftest_wait(static_cast<unsigned long long>(timeout_ms) * 1000000ull,

@@ -43,7 +43,32 @@ struct PrefillParams {
   unsigned long long timeout_ns;
 };
 
+// Everything the decode kernels need (see tilemix_decode_fwd).
+struct DecodeParams {
+  const void* q;             // fp16 [nseq][hq][d]
+  const void* k;             // fp16 [cache rows][hk][d]
+  const void* v;             // fp16 [cache rows][hk][d]
+  int8_t* k_i8;              // int8 [cache rows][hk][d] (last blocks rewritten)
+  float* k_scale;            // [hk][total_ktiles] (last blocks rewritten)
+  void* o;                   // fp16 [nseq][hq][d]
+  const int32_t* seq_start;  // [nseq]
+  const int32_t* seq_len;    // [nseq]
+  const int32_t* ktile_start;
+  const int32_t* qtile_start;
+  const uint64_t* masks;
+  const int32_t* g;
+  const int32_t* kv_head_of_q;
+  int8_t* q8;                // workspace: [nseq][hq][d] query codes
+  float* q_scale;            // workspace: [nseq][hq]
+  float* part_m;             // workspace: [nseq][hq][nsplit]
+  float* part_l;             // workspace: [nseq][hq][nsplit]
+  float* part_acc;           // workspace: [nseq][hq][nsplit][d]
+  int nseq, hq, hk, d, group, total_ktiles, nsplit, tiles_per_split;
+  float scale_log2;
+};
+
 // Launchers implemented in the CUDA translation unit.  Return cudaError_t.
+int launch_decode(const DecodeParams& p, cudaStream_t stream);
 // One launch quantises Q (128-row blocks) and K (64-row blocks); a null q or
 // k skips that side.  A non-null ticket is set to zero by the same launch
 // (the fused kernel that follows on the stream hands out work from it).
