@@ -175,19 +175,19 @@ def whole_job_tokens(tokens_per_rank, world):
     return int(tokens_per_rank) * int(world)
 
 
-def kernel_traffic(workload_name):
-    """DRAM bytes per launch of the fused kernel from the committed ncu record,
-    or None if the record is for another workload or the kernel source changed
-    since it was captured."""
+def kernel_traffic(workload_name, kernel="prefill_fwd_kernel<128>"):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or None
+    if the record is for another workload or one of the kernel's source files
+    changed since it was captured."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f)["prefill_fwd_kernel<128>"]
+            rec = json.load(f)[kernel]
         h = hashlib.sha256()
-        for name in ("tilemix_kernels.cu", "tilemix_ptx.cuh"):
+        for name in rec["sources"]:
             with open(os.path.join(ROOT, "tile_routed_mixed_b200", "csrc", name), "rb") as f:
                 h.update(f.read())
-        if rec["workload"] != workload_name or h.hexdigest()[:16] != rec["kernel_source_sha256_16"]:
+        if rec["workload"] != workload_name or h.hexdigest()[:16] != rec["sources_sha256_16"]:
             return None
         return float(rec["dram_bytes_per_launch"])
     except Exception:
@@ -440,6 +440,199 @@ def run_gpu(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ decode path ---
+
+DECODE_METRIC = "attention decode tok/s at 4k b8 (3B GQA shape), INT8 K cache; % of HBM roofline"
+
+
+def tile_starts(lengths):
+    """First query tile (128 rows) and key tile (64 keys) of each sequence."""
+    cq = np.zeros(len(lengths) + 1, dtype=np.int32)
+    ck = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cq[1:] = np.cumsum([(L + 127) // 128 for L in lengths])
+    ck[1:] = np.cumsum([(L + 63) // 64 for L in lengths])
+    return cq, ck
+
+
+def decode_bytes(lengths, hq, hk, d, masks, g):
+    """Algorithmic HBM bytes of one decode step, and of its split attention
+    kernel.  The step: every cached key once in its routed precision (INT8
+    codes or fp16), every cached value once (fp16), the K block re-quantised
+    (fp16 in, codes out), the new query rows and O.  The attention kernel: the
+    keys and values, and the query rows in fp16 and as codes (its partial
+    results are scratch and not counted)."""
+    cq, ck = tile_starts(lengths)
+    total = 0
+    requant = 0
+    for s, L in enumerate(lengths):
+        t = L - 1
+        nt = t // 64 + 1
+        for kv in range(hk):
+            w = int(masks[cq[s] + t // 128, kv])
+            for kt in range(nt):
+                keys = min(64, L - 64 * kt)
+                total += keys * d * (1 if (w >> (kt // int(g[s]))) & 1 else 2) + keys * d * 2
+            last = L - 64 * (t // 64)
+            requant += last * d * 3
+    attn = total + len(lengths) * hq * d * 3
+    return total + requant + len(lengths) * hq * d * 2 * 2, attn
+
+
+def run_decode(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference" and rank != 0:
+        return
+    w, lengths, g = workload(args.workload, args.template, args.percent)
+    hq, hk, d = w["hq"], w["hk"], w["d"]
+    if args.impl != "reference":
+        import torch
+        import torch.distributed as dist
+
+        import tile_routed_mixed_b200 as tm
+    cu = synth.cu_seqlens_of(lengths)
+    cq, ck = tile_starts(lengths)
+    if args.impl == "reference":
+        import oracle
+        masks, _, _ = oracle.build_routing(w["template"], w["percent"], w["routing_seed"],
+                                           lengths, hk, g, True)
+    else:
+        masks, _, _ = tm.tilemix_build_routing(w["template"], w["percent"], w["routing_seed"],
+                                               cu, hk, g, True)
+    T = int(cu[-1])
+    q, k, v = synth.make_qkv(rank, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
+    q_new = np.ascontiguousarray(q[cu[1:] - 1])          # the last position's query
+    nbytes, attn_bytes = decode_bytes(lengths, hq, hk, d, masks, g)
+    config = dict(bench_config(args, w, lengths, g), path="decode",
+                  l2="flush: 256 MB written before every step (the step moves %.0f MB)"
+                     % (nbytes / 1e6))
+    if args.impl == "reference":
+        if rank == 0:
+            t0 = time.perf_counter()
+            steps = 0
+            while steps < args.steps + args.warmup and (steps < 2 or time.perf_counter() - t0 < 60):
+                oracle.decode_rows(q_new, k, v, cu[:-1], lengths, masks, cq[:-1], g)
+                steps += 1
+            dt = (time.perf_counter() - t0) / steps
+            val = len(lengths) / dt
+            print(json.dumps({"impl": "reference", "metric": DECODE_METRIC, "value": val,
+                              "unit": "tok/s", "n_gpus": world, "steps": steps, "warmup": 0,
+                              "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+                              "vs_baseline": None, "dtype": "f16+i8", "data": "synthetic",
+                              "config": config,
+                              "cpu_baseline": {"value": val, "unit": "tok/s", "cores": host_cores(),
+                                               "kind": "oracle",
+                                               "sample": "%d full decode steps" % steps},
+                              "e2e": {"value": val, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+    kd, vd, qd = t(k), t(v), t(q_new)
+    k8 = torch.empty((T, hk, d), dtype=torch.int8, device=dev)
+    ks = torch.empty((hk, int(ck[-1])), dtype=torch.float32, device=dev)
+    cud, cqd, ckd = t(cu.astype(np.int32)), t(cq.astype(np.int32)), t(ck.astype(np.int32))
+    tm.tilemix_quantize_qk(None, kd, cud, cqd, ckd, len(lengths), T, int(cq[-1]), int(ck[-1]),
+                           hq, hk, d, None, None, k8, ks)     # the cache as prefill leaves it
+    dec = tm.TileMixDecode(cu[:-1], lengths, ck[:-1], cq[:-1], hq, hk, d, masks, g, int(ck[-1]),
+                           device=dev)
+    od = torch.empty_like(qd)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        dec(qd, kd, vd, k8, ks, od)
+    rc = tm.tilemix_get_error(stream)
+    if rc != tm.OK:
+        raise tm.TileMixError(rc, "warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in ev + kev:  # torch creates the CUDA event on first record: force it now
+        a.record(stream)
+        b.record(stream)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    for (a, b), e in zip(ev, kev):
+        flush.zero_()                     # the step's reads come from HBM, not L2
+        a.record(stream)
+        dec(qd, kd, vd, k8, ks, od, events=e)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    rc = tm.tilemix_get_error(stream)
+    if rc != tm.OK:
+        raise tm.TileMixError(rc, "timed steps")
+    per_step = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(per_step) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
+    ms, kern_ms = max_over_ranks([ms, kern_ms], device=dev)
+    # end to end: the new queries from pinned host memory in, O back out
+    qh = torch.from_numpy(q_new).pin_memory()
+    oh = torch.empty(q_new.shape, dtype=torch.float16).pin_memory()
+    n_e2e = max(args.steps // 4, 3)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_e2e)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev2:
+        flush.zero_()
+        a.record(stream)
+        qd.copy_(qh, non_blocking=True)
+        dec(qd, kd, vd, k8, ks, od)
+        oh.copy_(od, non_blocking=True)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in ev2) / n_e2e], device=dev)[0]
+    pk = peaks()
+    tokens = whole_job_tokens(len(lengths), world)
+    achieved = attn_bytes / (kern_ms / 1e3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": tokens / (ms / 1e3), "unit": "tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16+i8",
+        "data": "synthetic", "config": config,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"],
+                     "traffic": kernel_traffic(args.workload, "decode_attn_kernel<128>"),
+                     "kernel": "decode_attn_kernel<128>", "kernel_ms": kern_ms,
+                     "peak_kind": "copy bandwidth (%s)" % pk["source"],
+                     "algorithmic_bytes": attn_bytes, "step_bytes": nbytes,
+                     "step_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tok/s",
+                "h2d_bytes_per_step": int(q_new.nbytes), "d2h_bytes_per_step": int(q_new.nbytes)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        t0 = time.perf_counter()
+        n = 0
+        while n < 1 or time.perf_counter() - t0 < 10.0:
+            oracle.decode_rows(q_new, k, v, cu[:-1], lengths, masks, cq[:-1], g)
+            n += 1
+        dt = (time.perf_counter() - t0) / n
+        line["cpu_baseline"] = {"value": len(lengths) / dt, "unit": "tok/s", "cores": host_cores(),
+                                "kind": "oracle",
+                                "sample": "%d full decode steps of the workload" % n}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -450,10 +643,14 @@ def main():
     ap.add_argument("--template", default=None)
     ap.add_argument("--percent", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["prefill", "decode"], default="prefill",
+                    help="prefill (the headline metric) or the decode step with the INT8 K cache")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.path == "decode":
+        run_decode(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -257,6 +257,9 @@ typedef struct tilemix_decode_args {
   float softmax_scale;        /* 0 => 1 / sqrt(d) */
   void* workspace;            /* device, >= tilemix_decode_workspace_size(), 256-aligned */
   size_t workspace_bytes;
+  void* event_kernel_begin;   /* NULL, or a cudaEvent_t recorded on `stream` just before
+                                 the split attention kernel ... */
+  void* event_kernel_end;     /* ... and one recorded just after it (profiling) */
 } tilemix_decode_args;
 
 /* Bytes of device workspace tilemix_decode_fwd needs (query codes and the

@@ -64,6 +64,7 @@ class DecodeArgs(ctypes.Structure):
         ("hq", ctypes.c_int), ("hk", ctypes.c_int), ("d", ctypes.c_int),
         ("softmax_scale", ctypes.c_float),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("event_kernel_begin", ctypes.c_void_p), ("event_kernel_end", ctypes.c_void_p),
     ]
 
 

@@ -379,7 +379,9 @@ TILEMIX_API int tilemix_decode_fwd(const tilemix_decode_args* a, void* stream) {
   p.tiles_per_split = w.tiles_per_split;
   const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(a->d));
   p.scale_log2 = scale * 1.4426950408889634f;
-  if (tilemix::launch_decode(p, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (tilemix::launch_decode(p, static_cast<cudaStream_t>(stream),
+                             static_cast<cudaEvent_t>(a->event_kernel_begin),
+                             static_cast<cudaEvent_t>(a->event_kernel_end)) != cudaSuccess)
     return TILEMIX_ERR_CUDA;
   return TILEMIX_OK;
 }

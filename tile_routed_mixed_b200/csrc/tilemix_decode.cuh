@@ -304,17 +304,22 @@ __global__ void decode_combine_kernel(DecodeParams p) {
         __float2half_rn(l > 0.f ? o / l : 0.f);
 }
 
-int launch_decode(const DecodeParams& p, cudaStream_t stream) {
+int launch_decode(const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_begin,
+                  cudaEvent_t ev_end) {
   const unsigned prep_blocks = static_cast<unsigned>(p.nseq) * (p.hk + p.hq);
   decode_prep_kernel<<<prep_blocks, 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
+  if (ev_begin && (e = cudaEventRecord(ev_begin, stream)) != cudaSuccess)
+    return static_cast<int>(e);
   const unsigned attn_blocks = static_cast<unsigned>(p.nseq) * p.hk * p.nsplit;
   if (p.d == 128)
     decode_attn_kernel<128><<<attn_blocks, kDecodeThreads, 0, stream>>>(p);
   else
     decode_attn_kernel<64><<<attn_blocks, kDecodeThreads, 0, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return static_cast<int>(e);
+  if (ev_end && (e = cudaEventRecord(ev_end, stream)) != cudaSuccess)
+    return static_cast<int>(e);
   decode_combine_kernel<<<static_cast<unsigned>(p.nseq) * p.hq, 128, 0, stream>>>(p);
   return static_cast<int>(cudaGetLastError());
 }

@@ -68,7 +68,8 @@ struct DecodeParams {
 };
 
 // Launchers implemented in the CUDA translation unit.  Return cudaError_t.
-int launch_decode(const DecodeParams& p, cudaStream_t stream);
+int launch_decode(const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_begin,
+                  cudaEvent_t ev_end);
 // One launch quantises Q (128-row blocks) and K (64-row blocks); a null q or
 // k skips that side.  A non-null ticket is set to zero by the same launch
 // (the fused kernel that follows on the stream hands out work from it).

@@ -34,7 +34,7 @@ class TileMixDecode:
         self.kv_head_of_q = None if kv_head_of_q is None else to(kv_head_of_q, np.int32)
         self.workspace = None
 
-    def args(self, q, k, v, k_i8, k_scale, o):
+    def args(self, q, k, v, k_i8, k_scale, o, events=None):
         a = DecodeArgs()
         a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
         a.k_i8, a.k_scale, a.o = _ptr(k_i8), _ptr(k_scale), _ptr(o)
@@ -47,15 +47,18 @@ class TileMixDecode:
         a.softmax_scale = self.softmax_scale
         if self.workspace is not None:
             a.workspace, a.workspace_bytes = _ptr(self.workspace), self.workspace.numel()
+        if events is not None:  # (begin, end) torch.cuda.Event pair around the attention kernel
+            a.event_kernel_begin = events[0].cuda_event
+            a.event_kernel_end = events[1].cuda_event
         return a
 
-    def __call__(self, q, k, v, k_i8, k_scale, o=None, stream=None):
+    def __call__(self, q, k, v, k_i8, k_scale, o=None, stream=None, events=None):
         if o is None:
             o = torch.empty_like(q)
-        a = self.args(q, k, v, k_i8, k_scale, o)
+        a = self.args(q, k, v, k_i8, k_scale, o, events)
         need = tilemix_decode_workspace_size(a)
         if self.workspace is None or self.workspace.numel() < need:
             self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
-            a = self.args(q, k, v, k_i8, k_scale, o)
+            a = self.args(q, k, v, k_i8, k_scale, o, events)
         tilemix_decode_fwd(a, stream)
         return o
