@@ -233,9 +233,16 @@ int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
  *     current there (as tilemix_quantize_qk leaves them);
  *   - softmax state in fp32, P rounded to fp16 before P.V, O rounded once to
  *     fp16, as in the prefill path.
- * Three launches on `stream`: quantisation (last K blocks, query rows), split
- * attention over key ranges, merge.  Bad routing factors are reported by
- * tilemix_get_error() as for prefill. */
+ * One kernel launch on `stream` (after a memset of the workspace's split
+ * counters; K, V and the INT8 codes are read with TMA tile loads, so rows of
+ * a tile past seq_len[s] are read too, and zeros past cache_rows): each CTA
+ * takes tiles_per_split key tiles of one (sequence, KV
+ * head), quantises the new query rows of that KV head itself, re-quantises
+ * the last K block if its range holds it, and the CTA that finishes a
+ * (sequence, KV head) last merges the partial softmax states into O.  Bad
+ * routing factors, and a head map giving a KV head more than 16 query heads
+ * (only the first 16 are computed), are reported by tilemix_get_error() as
+ * for prefill. */
 typedef struct tilemix_decode_args {
   const void* q;              /* device fp16 [nseq][hq][d]: the new tokens' queries, 16-B aligned */
   const void* k;              /* device fp16 [cache_rows][hk][d], 16-B aligned */
@@ -253,22 +260,26 @@ typedef struct tilemix_decode_args {
   int nseq;                   /* >= 0 (0: nothing to do) */
   int max_seqlen;             /* >= every seq_len[s] (sizes the split of the key range) */
   int total_ktiles;           /* columns of k_scale */
+  int cache_rows;             /* rows of k, v and k_i8, >= every seq_start[s] + seq_len[s] */
   int hq, hk, d;              /* d in {64, 128}; hq % hk == 0; at most 16 query heads per KV head */
   float softmax_scale;        /* 0 => 1 / sqrt(d) */
+  int tiles_per_split;        /* 64-key tiles per CTA, >= 0; 0 => chosen from the SM
+                                 count (about four CTAs per resident slot) */
   void* workspace;            /* device, >= tilemix_decode_workspace_size(), 256-aligned */
   size_t workspace_bytes;
   void* event_kernel_begin;   /* NULL, or a cudaEvent_t recorded on `stream` just before
-                                 the split attention kernel ... */
+                                 the attention kernel ... */
   void* event_kernel_end;     /* ... and one recorded just after it (profiling) */
 } tilemix_decode_args;
 
-/* Bytes of device workspace tilemix_decode_fwd needs (query codes and the
- * split attention's partial states).  INVALID_ARG / UNSUPPORTED as for
+/* Bytes of device workspace tilemix_decode_fwd needs (the splits' partial
+ * softmax states and one counter per (sequence, KV head)).  INVALID_ARG / UNSUPPORTED as for
  * tilemix_decode_fwd. */
 int tilemix_decode_workspace_size(const tilemix_decode_args* args, size_t* bytes);
 
 /* Decode step as described above.  INVALID_ARG on a NULL required pointer, a
- * misaligned tensor, nseq < 0, max_seqlen < 1 or hq % hk != 0; UNSUPPORTED for
+ * misaligned tensor, nseq < 0, max_seqlen < 1, cache_rows < 1, tiles_per_split < 0
+ * or hq % hk != 0; UNSUPPORTED for
  * d not in {64, 128} or more than 16 query heads per KV head; WORKSPACE if the
  * workspace is missing, misaligned or too small; CUDA if a launch fails. */
 int tilemix_decode_fwd(const tilemix_decode_args* args, void* stream);

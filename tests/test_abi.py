@@ -148,7 +148,7 @@ def _fake_decode(**over):
     for f in ("q", "k", "v", "k_i8", "k_scale", "o", "seq_start", "seq_len", "ktile_start",
               "qtile_start", "masks", "g"):
         setattr(a, f, 4096)
-    a.nseq, a.max_seqlen, a.total_ktiles = 2, 300, 10
+    a.nseq, a.max_seqlen, a.total_ktiles, a.cache_rows = 2, 300, 10, 600
     a.hq, a.hk, a.d = 6, 2, 128
     for k, v in over.items():
         setattr(a, k, v)
@@ -169,6 +169,8 @@ def test_decode_argument_checks_are_synchronous():
         (dict(k_i8=None), tm.ERR_INVALID_ARG),
         (dict(q=4097), tm.ERR_INVALID_ARG),             # misaligned
         (dict(softmax_scale=-1.0), tm.ERR_INVALID_ARG),
+        (dict(tiles_per_split=-1), tm.ERR_INVALID_ARG),
+        (dict(cache_rows=0), tm.ERR_INVALID_ARG),
         (dict(workspace=None), tm.ERR_WORKSPACE),
         (dict(workspace=4096 + 128, workspace_bytes=1 << 30), tm.ERR_WORKSPACE),  # misaligned
     ]

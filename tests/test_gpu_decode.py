@@ -19,7 +19,7 @@ def _gpu():
     gc.set_test_timeout()
 
 
-def _run(lengths, hq, hk, d, masks_fn, g, seed, slack=37, kv_map=None):
+def _run(lengths, hq, hk, d, masks_fn, g, seed, slack=37, kv_map=None, tiles_per_split=0):
     import tile_routed_mixed_b200 as tm
     rng = np.random.default_rng(seed)
     nseq = len(lengths)
@@ -53,7 +53,7 @@ def _run(lengths, hq, hk, d, masks_fn, g, seed, slack=37, kv_map=None):
     dev = "cuda"
     t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
     dec = tm.TileMixDecode(starts, lengths, ktiles, qt[:-1], hq, hk, d, masks, g, total_kt,
-                           kv_head_of_q=kv_map, device=dev)
+                           kv_head_of_q=kv_map, device=dev, tiles_per_split=tiles_per_split)
     qd, kd, vd, k8d, ksd = t(q), t(k), t(v), t(k8), t(ks)
     o = dec(qd, kd, vd, k8d, ksd)
     torch.cuda.synchronize()
@@ -109,3 +109,23 @@ def test_decode_long_context():
     lengths = [16384, 5000]
     g = np.array([oracle.auto_g(L) for L in lengths], dtype=np.int32)
     _run(lengths, 8, 2, 128, _template("row_random", 25, lengths, 2, g), g, seed=9)
+
+
+@pytest.mark.parametrize("group,d", [(1, 128), (2, 64), (5, 128), (7, 64), (8, 128), (12, 64),
+                                     (16, 128)])
+def test_decode_group_sizes(group, d):
+    """Every compiled group size, and the generic path (12, 16) that takes any
+    count up to 16."""
+    lengths = [70, 257, 1]
+    g = np.ones(len(lengths), dtype=np.int32)
+    _run(lengths, 2 * group, 2, d, _template("sptrans", 75, lengths, 2, g), g, seed=10 + group)
+
+
+@pytest.mark.parametrize("tps", [1, 3, 5, 16, 64])
+def test_decode_tiles_per_split(tps):
+    """Splits of several tiles: the copy ring wraps (tiles past the number of
+    stages), splits end ragged, and one split may hold a whole sequence."""
+    lengths = [1000, 64, 3000, 129]
+    g = np.ones(len(lengths), dtype=np.int32)
+    _run(lengths, 12, 4, 128, _template("sptrans", 75, lengths, 4, g), g, seed=30 + tps,
+         tiles_per_split=tps)

@@ -61,8 +61,9 @@ class DecodeArgs(ctypes.Structure):
         ("ktile_start", ctypes.c_void_p), ("qtile_start", ctypes.c_void_p),
         ("masks", ctypes.c_void_p), ("g", ctypes.c_void_p), ("kv_head_of_q", ctypes.c_void_p),
         ("nseq", ctypes.c_int), ("max_seqlen", ctypes.c_int), ("total_ktiles", ctypes.c_int),
+        ("cache_rows", ctypes.c_int),
         ("hq", ctypes.c_int), ("hk", ctypes.c_int), ("d", ctypes.c_int),
-        ("softmax_scale", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float), ("tiles_per_split", ctypes.c_int),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("event_kernel_begin", ctypes.c_void_p), ("event_kernel_end", ctypes.c_void_p),
     ]

@@ -274,7 +274,7 @@ TILEMIX_API int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, vo
 namespace {
 
 struct DecodeLayout {
-  size_t q8, q_scale, part_m, part_l, part_acc, total;
+  size_t part_m, part_l, part_acc, counters, total;
   int nsplit, tiles_per_split;
 };
 
@@ -283,7 +283,9 @@ int check_decode(const tilemix_decode_args* a) {
   if (a->d != 64 && a->d != 128) return TILEMIX_ERR_UNSUPPORTED;
   if (a->hq < 1 || a->hk < 1 || a->hq % a->hk != 0) return TILEMIX_ERR_INVALID_ARG;
   if (a->kv_head_of_q == nullptr && a->hq / a->hk > 16) return TILEMIX_ERR_UNSUPPORTED;
-  if (a->nseq < 0 || a->max_seqlen < 1 || a->total_ktiles < 0) return TILEMIX_ERR_INVALID_ARG;
+  if (a->nseq < 0 || a->max_seqlen < 1 || a->total_ktiles < 0 || a->tiles_per_split < 0 ||
+      a->cache_rows < 1)
+    return TILEMIX_ERR_INVALID_ARG;
   if (!(a->softmax_scale >= 0.f) || std::isinf(a->softmax_scale)) return TILEMIX_ERR_INVALID_ARG;
   if (a->nseq == 0) return TILEMIX_OK;
   if (!a->q || !a->k || !a->v || !a->k_i8 || !a->k_scale || !a->o || !a->seq_start ||
@@ -303,29 +305,30 @@ int decode_sms() {
   return sms;
 }
 
-// The key range of every (sequence, KV head) is cut into nsplit pieces so that
-// about two CTAs per SM run the attention step.
+// The key range of every (sequence, KV head) is cut into splits of
+// tiles_per_split key tiles, one CTA each: small enough that the grid holds
+// about four CTAs per resident slot (two per SM), so the tail of the launch
+// is short, and no smaller than one tile.
 DecodeLayout decode_layout(const tilemix_decode_args* a) {
   DecodeLayout w{};
   const int max_tiles = (a->max_seqlen + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N;
-  const long long units = static_cast<long long>(a->nseq) * a->hk;
-  long long ns = units > 0 ? (2LL * decode_sms() + units - 1) / units : 1;
-  if (ns < 1) ns = 1;
-  if (ns > max_tiles) ns = max_tiles;
-  w.nsplit = static_cast<int>(ns);
-  w.tiles_per_split = (max_tiles + w.nsplit - 1) / w.nsplit;
+  const long long tiles = static_cast<long long>(a->nseq) * a->hk * max_tiles;
+  long long per = a->tiles_per_split > 0 ? a->tiles_per_split : tiles / (8LL * decode_sms());
+  if (per < 1) per = 1;
+  if (a->tiles_per_split == 0 && per > 16) per = 16;
+  if (per > max_tiles) per = max_tiles;
+  w.tiles_per_split = static_cast<int>(per);
+  w.nsplit = (max_tiles + w.tiles_per_split - 1) / w.tiles_per_split;
   const size_t rows = static_cast<size_t>(a->nseq) * a->hq;
   size_t off = 0;
-  w.q8 = off;
-  off = round_up(off + rows * a->d, 256);
-  w.q_scale = off;
-  off = round_up(off + rows * sizeof(float), 256);
   w.part_m = off;
   off = round_up(off + rows * w.nsplit * sizeof(float), 256);
   w.part_l = off;
   off = round_up(off + rows * w.nsplit * sizeof(float), 256);
   w.part_acc = off;
   off = round_up(off + rows * w.nsplit * a->d * sizeof(float), 256);
+  w.counters = off;
+  off = round_up(off + static_cast<size_t>(a->nseq) * a->hk * sizeof(int), 256);
   w.total = off;
   return w;
 }
@@ -351,6 +354,18 @@ TILEMIX_API int tilemix_decode_fwd(const tilemix_decode_args* a, void* stream) {
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   tilemix::DecodeParams p;
   std::memset(&p, 0, sizeof(p));
+  const int d = a->d, rows = a->cache_rows;
+  if ((rc = encode_rows(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, a->hk, d, 64,
+                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_k8, a->k_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, a->hk, d, d,
+                        TILEMIX_BLOCK_N,
+                        d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B)) !=
+      TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, a->hk, d, 64,
+                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
   p.q = a->q;
   p.k = a->k;
   p.v = a->v;
@@ -364,11 +379,10 @@ TILEMIX_API int tilemix_decode_fwd(const tilemix_decode_args* a, void* stream) {
   p.masks = a->masks;
   p.g = a->g;
   p.kv_head_of_q = a->kv_head_of_q;
-  p.q8 = reinterpret_cast<int8_t*>(ws + w.q8);
-  p.q_scale = reinterpret_cast<float*>(ws + w.q_scale);
   p.part_m = reinterpret_cast<float*>(ws + w.part_m);
   p.part_l = reinterpret_cast<float*>(ws + w.part_l);
   p.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
+  p.counters = reinterpret_cast<int*>(ws + w.counters);
   p.nseq = a->nseq;
   p.hq = a->hq;
   p.hk = a->hk;
@@ -377,6 +391,8 @@ TILEMIX_API int tilemix_decode_fwd(const tilemix_decode_args* a, void* stream) {
   p.total_ktiles = a->total_ktiles;
   p.nsplit = w.nsplit;
   p.tiles_per_split = w.tiles_per_split;
+  p.gcap = !a->kv_head_of_q && a->hq / a->hk <= 8 ? a->hq / a->hk : 16;
+  p.timeout_ns = wait_timeout_ns();
   const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(a->d));
   p.scale_log2 = scale * 1.4426950408889634f;
   if (tilemix::launch_decode(p, static_cast<cudaStream_t>(stream),

@@ -45,6 +45,9 @@ struct PrefillParams {
 
 // Everything the decode kernels need (see tilemix_decode_fwd).
 struct DecodeParams {
+  CUtensorMap tm_k;          // fp16 K   [cache rows][hk][d], box {64, 1, 64}, 128B swizzle
+  CUtensorMap tm_k8;         // int8 K   [cache rows][hk][d], box {d, 1, 64}
+  CUtensorMap tm_v;          // fp16 V   [cache rows][hk][d], box {64, 1, 64}, 128B swizzle
   const void* q;             // fp16 [nseq][hq][d]
   const void* k;             // fp16 [cache rows][hk][d]
   const void* v;             // fp16 [cache rows][hk][d]
@@ -58,13 +61,14 @@ struct DecodeParams {
   const uint64_t* masks;
   const int32_t* g;
   const int32_t* kv_head_of_q;
-  int8_t* q8;                // workspace: [nseq][hq][d] query codes
-  float* q_scale;            // workspace: [nseq][hq]
   float* part_m;             // workspace: [nseq][hq][nsplit]
   float* part_l;             // workspace: [nseq][hq][nsplit]
   float* part_acc;           // workspace: [nseq][hq][nsplit][d]
+  int* counters;             // workspace: [nseq][hk] finished splits (zeroed per call)
   int nseq, hq, hk, d, group, total_ktiles, nsplit, tiles_per_split;
+  int gcap;                  // query heads one CTA holds (hq / hk, or 16 with a head map)
   float scale_log2;
+  unsigned long long timeout_ns;
 };
 
 // Launchers implemented in the CUDA translation unit.  Return cudaError_t.

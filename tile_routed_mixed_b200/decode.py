@@ -16,7 +16,8 @@ class TileMixDecode:
     qtile_start[s] of masks ([total_qtiles, hk])."""
 
     def __init__(self, seq_start, seq_len, ktile_start, qtile_start, hq, hk, d, masks, g,
-                 total_ktiles, softmax_scale=0.0, kv_head_of_q=None, device="cuda"):
+                 total_ktiles, softmax_scale=0.0, kv_head_of_q=None, device="cuda",
+                 tiles_per_split=0):
         self.device = torch.device(device)
         to = lambda a, dt: torch.as_tensor(np.ascontiguousarray(a, dtype=dt)).to(self.device)
         self.seq_len_h = [int(x) for x in seq_len]
@@ -25,6 +26,7 @@ class TileMixDecode:
         self.max_seqlen = max(self.seq_len_h) if self.seq_len_h else 1
         self.total_ktiles = int(total_ktiles)
         self.softmax_scale = float(softmax_scale)
+        self.tiles_per_split = int(tiles_per_split)
         self.seq_start = to(seq_start, np.int32)
         self.seq_len = to(seq_len, np.int32)
         self.ktile_start = to(ktile_start, np.int32)
@@ -43,8 +45,10 @@ class TileMixDecode:
         a.masks, a.g = _ptr(self.masks), _ptr(self.g)
         a.kv_head_of_q = _ptr(self.kv_head_of_q) if self.kv_head_of_q is not None else None
         a.nseq, a.max_seqlen, a.total_ktiles = self.nseq, self.max_seqlen, self.total_ktiles
+        a.cache_rows = int(k.shape[0]) if k is not None else 0
         a.hq, a.hk, a.d = self.hq, self.hk, self.d
         a.softmax_scale = self.softmax_scale
+        a.tiles_per_split = self.tiles_per_split
         if self.workspace is not None:
             a.workspace, a.workspace_bytes = _ptr(self.workspace), self.workspace.numel()
         if events is not None:  # (begin, end) torch.cuda.Event pair around the attention kernel
