@@ -263,8 +263,8 @@ typedef struct tilemix_decode_args {
   int cache_rows;             /* rows of k, v and k_i8, >= every seq_start[s] + seq_len[s] */
   int hq, hk, d;              /* d in {64, 128}; hq % hk == 0; at most 16 query heads per KV head */
   float softmax_scale;        /* 0 => 1 / sqrt(d) */
-  int tiles_per_split;        /* 64-key tiles per CTA, >= 0; 0 => chosen from the SM
-                                 count (about four CTAs per resident slot) */
+  int tiles_per_split;        /* 64-key tiles per CTA, >= 0; 0 => chosen so that the
+                                 CTAs fill the resident slots (two per SM) about once */
   void* workspace;            /* device, >= tilemix_decode_workspace_size(), 256-aligned */
   size_t workspace_bytes;
   void* event_kernel_begin;   /* NULL, or a cudaEvent_t recorded on `stream` just before

@@ -305,17 +305,21 @@ int decode_sms() {
   return sms;
 }
 
-// The key range of every (sequence, KV head) is cut into splits of
-// tiles_per_split key tiles, one CTA each: small enough that the grid holds
-// about four CTAs per resident slot (two per SM), so the tail of the launch
-// is short, and no smaller than one tile.
+// The key range of every (sequence, KV head) is cut into nsplit splits of
+// tiles_per_split key tiles, one CTA each, so that the grid fills the
+// resident slots (two CTAs per SM) about once: fewer, longer splits pay the
+// per-CTA start (metadata, query rows) and merge less often.
 DecodeLayout decode_layout(const tilemix_decode_args* a) {
   DecodeLayout w{};
   const int max_tiles = (a->max_seqlen + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N;
-  const long long tiles = static_cast<long long>(a->nseq) * a->hk * max_tiles;
-  long long per = a->tiles_per_split > 0 ? a->tiles_per_split : tiles / (8LL * decode_sms());
+  long long per = a->tiles_per_split;
+  if (per <= 0) {
+    const long long units = static_cast<long long>(a->nseq) * a->hk;
+    long long ns = units > 0 ? 2LL * decode_sms() / units : 1;
+    if (ns < 1) ns = 1;
+    per = (max_tiles + ns - 1) / ns;
+  }
   if (per < 1) per = 1;
-  if (a->tiles_per_split == 0 && per > 16) per = 16;
   if (per > max_tiles) per = max_tiles;
   w.tiles_per_split = static_cast<int>(per);
   w.nsplit = (max_tiles + w.tiles_per_split - 1) / w.tiles_per_split;
@@ -391,7 +395,6 @@ TILEMIX_API int tilemix_decode_fwd(const tilemix_decode_args* a, void* stream) {
   p.total_ktiles = a->total_ktiles;
   p.nsplit = w.nsplit;
   p.tiles_per_split = w.tiles_per_split;
-  p.gcap = !a->kv_head_of_q && a->hq / a->hk <= 8 ? a->hq / a->hk : 16;
   p.timeout_ns = wait_timeout_ns();
   const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(a->d));
   p.scale_log2 = scale * 1.4426950408889634f;

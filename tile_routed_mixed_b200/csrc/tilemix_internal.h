@@ -66,7 +66,6 @@ struct DecodeParams {
   float* part_acc;           // workspace: [nseq][hq][nsplit][d]
   int* counters;             // workspace: [nseq][hk] finished splits (zeroed per call)
   int nseq, hq, hk, d, group, total_ktiles, nsplit, tiles_per_split;
-  int gcap;                  // query heads one CTA holds (hq / hk, or 16 with a head map)
   float scale_log2;
   unsigned long long timeout_ns;
 };
