@@ -512,3 +512,134 @@ def test_decode_query_rows_are_their_own_blocks():
     c, s = oracle.quantize_rows(x)
     assert list(c[0, 0, :3]) == [127, -64, 0] and s[0, 0] == np.float32(1.0)
     assert c[1, 0, 0] == 127 and s[1, 0] == np.float32(np.float32(2.0) / np.float32(127.0))
+
+
+# ---------------------------------------------------------- adaptive routing --
+# Pins of oracle/adaptive.py (the pooled-score policy): hand-derived fp32
+# values for the stated summation order, closed-form words for constructed
+# inputs, the static templates' quota, and the aligned-sparse layout that the
+# policy must reproduce when the scores grow with the key position.
+
+from oracle import adaptive as ad  # noqa: E402
+
+
+def test_adaptive_mean_uses_interleaved_partial_sums():
+    # item 0 = 2^24, items 1 and 9 = 1: partial sum 1 holds 1 + 1 = 2 exactly,
+    # so the total is 2^24 + 2; a running sum would lose both ones (ties to even)
+    items = np.zeros((10, 1), dtype=np.float32)
+    items[0, 0] = 2.0 ** 24
+    items[1, 0] = 1.0
+    items[9, 0] = 1.0
+    got = ad.interleaved_mean(items)
+    assert got.dtype == np.float32
+    assert got[0] == np.float32(16777218.0) / np.float32(10.0)
+    seq = np.float32(0.0)
+    for x in items[:, 0]:
+        seq = np.float32(seq + x)
+    assert seq == np.float32(2.0 ** 24)      # what the order rules out
+    assert np.array_equal(ad.interleaved_mean(np.zeros((0, 3), np.float32)), np.zeros(3, np.float32))
+    # exact small integers: the mean is exact
+    v = np.arange(24, dtype=np.float32).reshape(24, 1)
+    assert ad.interleaved_mean(v)[0] == np.float32(11.5)
+
+
+def test_adaptive_dot_rounds_each_product():
+    a = np.float32(1.0 + 2.0 ** -12)
+    # a*a = 1 + 2^-11 + 2^-24 rounds to 1 + 2^-11 (tie to even); a*(-a) the
+    # same with a minus sign: separately rounded the dot is 0, a fused
+    # multiply-add in the second step would give -2^-24
+    got = ad.ordered_dot(np.array([a, a], np.float32), np.array([[a, -a]], np.float32))
+    assert got[0] == np.float32(0.0)
+    assert math.copysign(1.0, float(np.float32(a) * np.float32(a) - np.float64(a) * np.float64(a))) < 0
+
+
+def test_adaptive_choose_ties_go_to_the_lower_group():
+    assert ad.choose_int8([0.0] * 6, 3) == {0, 1, 2}
+    assert ad.choose_int8([3.0, 1.0, 1.0, 2.0], 2) == {1, 2}
+    assert ad.choose_int8([3.0, 1.0, 1.0, 2.0], 3) == {1, 2, 3}
+    assert ad.choose_int8([1.0, -0.0, 0.0], 1) == {1}  # -0 == 0: the lower index
+
+
+def _ramp_keys(lengths, hk, d, slope):
+    """K rows whose channel 0 holds slope * (key tile index + 1), other channels 0."""
+    T = sum(lengths)
+    k = np.zeros((T, hk, d), dtype=np.float16)
+    start = 0
+    for L in lengths:
+        for j in range(L):
+            k[start + j, :, 0] = np.float16(slope * (j // 64 + 1))
+        start += L
+    return k
+
+
+@pytest.mark.parametrize("percent", [0, 25, 50, 75, 100])
+def test_adaptive_rising_scores_give_the_aligned_sparse_layout(percent):
+    # q = e0 and k tiles rising along the key axis: the score grows with the
+    # tile, so each row's lowest-scoring groups are its leftmost ones and the
+    # FP16 groups are the rightmost f_r: the aligned-sparse template's words
+    lengths, hq, hk, d = [300, 1000, 64], 4, 2, 64
+    T = sum(lengths)
+    q = np.zeros((T, hq, d), dtype=np.float16)
+    q[:, :, 0] = np.float16(0.5)
+    k = _ramp_keys(lengths, hk, d, 0.25)
+    g = [1, 2, 1]
+    for causal in (True, False):
+        got = ad.route_pooled(q, k, lengths, hq, hk, g, causal, percent)
+        want, _, _ = oracle.build_routing("aligned_sparse", percent, 0, lengths, hk, g, causal)
+        assert np.array_equal(got, want), (percent, causal)
+
+
+def test_adaptive_falling_scores_keep_the_left_groups():
+    # scores falling along the key axis: the INT8 groups are the rightmost k_r
+    lengths, hq, hk, d = [1000], 2, 1, 64
+    q = np.zeros((1000, hq, d), dtype=np.float16)
+    q[:, :, 0] = np.float16(-1.0)
+    k = _ramp_keys(lengths, hk, d, 0.125)
+    got = ad.route_pooled(q, k, lengths, hq, hk, [1], True, 50)
+    n = [oracle.legal_groups(qt, 1000, 1, True) for qt in range(oracle.n_qtiles(1000))]
+    kq = ad._quota(n, 50)
+    for qt, (x, kr) in enumerate(zip(n, kq)):
+        want = sum(1 << b for b in range(x - kr, x))
+        assert int(got[qt, 0]) == want, qt
+
+
+@pytest.mark.parametrize("percent", [10, 33, 75])
+def test_adaptive_quota_and_legality(percent):
+    rng = np.random.default_rng(7)
+    lengths, hq, hk, d = [129, 777, 2048], 6, 2, 64
+    T = sum(lengths)
+    q = rng.standard_normal((T, hq, d)).astype(np.float16)
+    k = rng.standard_normal((T, hk, d)).astype(np.float16)
+    g = [1, 1, 2]
+    got = ad.route_pooled(q, k, lengths, hq, hk, g, True, percent)
+    cq = 0
+    for s, L in enumerate(lengths):
+        n = [oracle.legal_groups(qt, L, g[s], True) for qt in range(oracle.n_qtiles(L))]
+        kq = ad._quota(n, percent)
+        for qt, (x, kr) in enumerate(zip(n, kq)):
+            for kv in range(hk):
+                w = int(got[cq + qt, kv])
+                assert w >> x == 0                      # no bits past the legal groups
+                assert bin(w).count("1") == kr          # the templates' per-row quota
+        assert sum(kq) == oracle.int8_target(percent, sum(n))
+        cq += oracle.n_qtiles(L)
+
+
+def test_adaptive_pooled_means_by_brute_force():
+    rng = np.random.default_rng(3)
+    lengths, hq, hk, d = [130, 64], 6, 2, 64
+    T = sum(lengths)
+    q = rng.standard_normal((T, hq, d)).astype(np.float16)
+    k = rng.standard_normal((T, hk, d)).astype(np.float16)
+    kv_map = np.array([1, 0, 0, 1, 1, 0], dtype=np.int32)
+    qb, kb = ad.pooled_means(q, k, lengths, hq, hk, kv_map)
+    assert qb.shape == (3, hk, d) and kb.shape == (4, hk, d)
+    # q tile 1 of sequence 0 is rows 128..129 of heads {1, 2, 5} for KV head 0
+    items = [q[r, h].astype(np.float64) for h in (1, 2, 5) for r in (128, 129)]
+    np.testing.assert_allclose(qb[1, 0], np.mean(items, axis=0), rtol=1e-6, atol=1e-6)
+    # key tile 2 of sequence 0 is rows 128..129
+    np.testing.assert_allclose(kb[2, 1], k[128:130, 1].astype(np.float64).mean(axis=0),
+                               rtol=1e-6, atol=1e-6)
+    # key tile 3 is the 64 rows of sequence 1
+    np.testing.assert_allclose(kb[3, 0], k[130:194, 0].astype(np.float64).mean(axis=0),
+                               rtol=1e-5, atol=1e-6)
