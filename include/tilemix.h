@@ -284,6 +284,64 @@ int tilemix_decode_workspace_size(const tilemix_decode_args* args, size_t* bytes
  * workspace is missing, misaligned or too small; CUDA if a launch fails. */
 int tilemix_decode_fwd(const tilemix_decode_args* args, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Content-aware (adaptive) routing through the same routing words.
+ *
+ * The pages say the mask interface can take adaptive policies and evaluate
+ * none ("TileMix: Tile-Centric Mixed-Precision Attention for LLM Inference
+ * Acceleration", agihunt.info summary, limitations paragraph; "Precision Has
+ * a Map: TileMix Routes INT8 Inside Dense Attention", cognaptus.com,
+ * "Placement can matter more than the nominal percentage").  This library's
+ * policy, pooled scores:
+ *   - for query-tile row r of sequence s and KV head kv, qbar = the mean of q
+ *     over the row's valid query rows and kv's query heads, kbar_kt = the mean
+ *     of k over key tile kt's valid keys;
+ *   - each legal key tile kt scores qbar . kbar_kt, each legal group the
+ *     highest score of its tiles;
+ *   - the row's k_r lowest-scoring groups are INT8 (ties: the lower group),
+ *     k_r from the proportional quota of the static templates (floor(p n_r /
+ *     100), the sequence's leftover to the rows with the largest remainder,
+ *     ties to the lower row), so each sequence gets the templates' INT8 count;
+ *   - fp32 in a fixed order: a mean sums its items (q head-major, heads
+ *     ascending, then rows ascending; k rows ascending) into 8 interleaved
+ *     partial sums (item m into sum m mod 8), adds them in order 0..7 and
+ *     divides by the count (no items: zero); a dot adds the separately
+ *     rounded products over channels ascending.  The words are reproducible
+ *     bit for bit.
+ * Output: masks[total_qtiles][hk] on the device, the layout
+ * tilemix_build_routing writes; bits past a row's legal groups are 0.
+ * Three launches on `stream` (query means, key means, words). */
+typedef struct tilemix_route_args {
+  const void* q;              /* device fp16 [T][hq][d], 16-B aligned */
+  const void* k;              /* device fp16 [T][hk][d], 16-B aligned */
+  const int32_t* cu_seqlens_h;/* host [nseq + 1]: validation and grid sizes */
+  const int32_t* g_h;         /* host [nseq]: routing-group factors */
+  const int32_t* cu_seqlens;  /* device copies of the same values ... */
+  const int32_t* cu_qtiles;   /* ... and the tile offsets (tilemix_tile_offsets) */
+  const int32_t* cu_ktiles;
+  const int32_t* g;
+  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk) */
+  int nseq, hq, hk, d;        /* d in {64, 128}; at most 256 query heads per KV head */
+  int causal;                 /* 0 or 1 */
+  int int8_percent;           /* 0..100 */
+  uint64_t* masks;            /* device out [total_qtiles][hk] */
+  void* workspace;            /* device, >= tilemix_route_workspace_size(), 256-aligned */
+  size_t workspace_bytes;
+  void* event_begin;          /* NULL, or cudaEvent_t recorded before the launches ... */
+  void* event_end;            /* ... and after them (profiling) */
+} tilemix_route_args;
+
+/* Bytes of workspace tilemix_route_pooled needs (the fp32 means). */
+int tilemix_route_workspace_size(const tilemix_route_args* args, size_t* bytes);
+
+/* Pooled-score routing as described above.  INVALID_ARG on a NULL required
+ * pointer, a misaligned tensor, a bad percent, causal flag or g, lengths that
+ * do not start at 0 or decrease, a row with more than 64 groups, or hq % hk
+ * != 0 without a head map; UNSUPPORTED for d not in {64, 128} or more than 256
+ * query heads per KV head; WORKSPACE for a missing or small workspace; CUDA
+ * if a launch fails.  All argument errors are returned before any launch. */
+int tilemix_route_pooled(const tilemix_route_args* args, void* stream);
+
 /* Self test of the failure path: enqueues one warp that waits on a device
  * barrier nothing ever signals, with the same bounded wait the attention
  * kernel uses, limited to timeout_ms (1..10000).  The wait gives up, latches

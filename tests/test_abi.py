@@ -178,3 +178,59 @@ def test_decode_argument_checks_are_synchronous():
         assert L.tilemix_decode_fwd(ctypes.byref(_fake_decode(**over)), None) == want, over
     # nothing to do: OK without touching any pointer
     assert L.tilemix_decode_fwd(ctypes.byref(_fake_decode(nseq=0, q=None)), None) == tm.OK
+
+
+def _fake_route(cu, g, **over):
+    a = tm.RouteArgs()
+    for f in ("q", "k", "cu_seqlens", "cu_qtiles", "cu_ktiles", "g", "masks"):
+        setattr(a, f, 4096)
+    a.cu_seqlens_h = cu.ctypes.data_as(ctypes.c_void_p)
+    a.g_h = g.ctypes.data_as(ctypes.c_void_p)
+    a.nseq, a.hq, a.hk, a.d, a.causal, a.int8_percent = len(g), 6, 2, 128, 1, 50
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_route_argument_checks_are_synchronous():
+    """Every argument error of tilemix_route_pooled returns before any launch
+    (fake device pointers; nothing is dereferenced on these paths)."""
+    L = ctypes.CDLL(tm.LIB_PATH)
+    L.tilemix_route_pooled.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    L.tilemix_route_workspace_size.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    cu = np.array([0, 300, 1300], dtype=np.int32)
+    g = np.array([1, 1], dtype=np.int32)
+    n = ctypes.c_size_t(0)
+    assert L.tilemix_route_workspace_size(ctypes.byref(_fake_route(cu, g)), ctypes.byref(n)) == tm.OK
+    # 3 + 8 query tiles and 5 + 16 key tiles, 2 KV heads, d 128, fp32 means
+    assert n.value == (11 * 2 * 128 * 4 + 255) // 256 * 256 + (21 * 2 * 128 * 4 + 255) // 256 * 256
+    long_seq = np.array([0, 64 * 64 + 1], dtype=np.int32)   # 65 groups at g = 1
+    cases = [
+        (dict(d=80), tm.ERR_UNSUPPORTED),
+        (dict(int8_percent=101), tm.ERR_INVALID_ARG),
+        (dict(int8_percent=-1), tm.ERR_INVALID_ARG),
+        (dict(causal=2), tm.ERR_INVALID_ARG),
+        (dict(hq=6, hk=4), tm.ERR_INVALID_ARG),
+        (dict(hq=600, hk=2), tm.ERR_UNSUPPORTED),
+        (dict(q=None), tm.ERR_INVALID_ARG),
+        (dict(k=4100), tm.ERR_INVALID_ARG),            # misaligned
+        (dict(masks=4100), tm.ERR_INVALID_ARG),        # not 8-byte aligned
+        (dict(cu_seqlens_h=None), tm.ERR_INVALID_ARG),
+        (dict(workspace=None), tm.ERR_WORKSPACE),
+        (dict(workspace=4096 + 64, workspace_bytes=1 << 30), tm.ERR_WORKSPACE),
+    ]
+    for over, want in cases:
+        assert L.tilemix_route_pooled(ctypes.byref(_fake_route(cu, g, **over)), None) == want, over
+    bad_g = np.array([1, 0], dtype=np.int32)
+    assert L.tilemix_route_pooled(ctypes.byref(_fake_route(cu, bad_g)), None) == tm.ERR_INVALID_ARG
+    one = np.array([1], dtype=np.int32)
+    assert L.tilemix_route_pooled(ctypes.byref(_fake_route(long_seq, one)), None) == tm.ERR_INVALID_ARG
+    two = np.array([2], dtype=np.int32)                    # g = 2 brings it to 33 groups
+    a = _fake_route(long_seq, two, workspace=None)
+    assert L.tilemix_route_pooled(ctypes.byref(a), None) == tm.ERR_WORKSPACE
+    dec = np.array([0, 300, 200], dtype=np.int32)          # decreasing offsets
+    assert L.tilemix_route_pooled(ctypes.byref(_fake_route(dec, g)), None) == tm.ERR_INVALID_ARG
+    empty = np.array([0], dtype=np.int32)
+    a = _fake_route(empty, np.zeros(0, np.int32), q=None, k=None)
+    a.nseq = 0
+    assert L.tilemix_route_pooled(ctypes.byref(a), None) == tm.OK

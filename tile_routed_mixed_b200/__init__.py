@@ -69,6 +69,21 @@ class DecodeArgs(ctypes.Structure):
     ]
 
 
+class RouteArgs(ctypes.Structure):
+    """Mirror of ``tilemix_route_args``."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
+        ("cu_seqlens_h", ctypes.c_void_p), ("g_h", ctypes.c_void_p),
+        ("cu_seqlens", ctypes.c_void_p), ("cu_qtiles", ctypes.c_void_p),
+        ("cu_ktiles", ctypes.c_void_p), ("g", ctypes.c_void_p), ("kv_head_of_q", ctypes.c_void_p),
+        ("nseq", ctypes.c_int), ("hq", ctypes.c_int), ("hk", ctypes.c_int), ("d", ctypes.c_int),
+        ("causal", ctypes.c_int), ("int8_percent", ctypes.c_int),
+        ("masks", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("event_begin", ctypes.c_void_p), ("event_end", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -104,6 +119,11 @@ def lib():
                                                     ctypes.POINTER(ctypes.c_size_t)]
         L.tilemix_decode_fwd.restype = I
         L.tilemix_decode_fwd.argtypes = [ctypes.POINTER(DecodeArgs), P]
+        L.tilemix_route_workspace_size.restype = I
+        L.tilemix_route_workspace_size.argtypes = [ctypes.POINTER(RouteArgs),
+                                                   ctypes.POINTER(ctypes.c_size_t)]
+        L.tilemix_route_pooled.restype = I
+        L.tilemix_route_pooled.argtypes = [ctypes.POINTER(RouteArgs), P]
         L.tilemix_selftest_wait_timeout.restype = I
         L.tilemix_selftest_wait_timeout.argtypes = [I, P]
         L.tilemix_get_error.restype = I
@@ -266,11 +286,63 @@ def tilemix_decode_fwd(args: DecodeArgs, stream=None):
            "tilemix_decode_fwd")
 
 
+def tilemix_route_workspace_size(args: RouteArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tilemix_route_workspace_size(ctypes.byref(args), ctypes.byref(n)),
+           "tilemix_route_workspace_size")
+    return int(n.value)
+
+
+def tilemix_route_pooled(args: RouteArgs, stream=None):
+    _check(lib().tilemix_route_pooled(ctypes.byref(args), _stream_handle(stream)),
+           "tilemix_route_pooled")
+
+
+def route_pooled(q, k, lengths, hq, hk, g, causal, int8_percent, kv_head_of_q=None,
+                 stream=None, events=None, workspace=None):
+    """Pooled-score routing words [total_qtiles, hk] (int64 view of uint64) on
+    q's device for the packed batch ``lengths``."""
+    import numpy as np
+    import torch
+    dev = q.device
+    lengths = [int(x) for x in lengths]
+    cu = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lengths)
+    cq, ck = tilemix_tile_offsets(cu)
+    gh = np.ascontiguousarray(np.asarray(g, dtype=np.int32))
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    cud, cqd, ckd, gd = to(cu), to(cq), to(ck), to(gh)
+    masks = torch.empty((int(cq[-1]), int(hk)), dtype=torch.int64, device=dev)
+    a = RouteArgs()
+    a.q, a.k = _ptr(q), _ptr(k)
+    a.cu_seqlens_h = cu.ctypes.data_as(ctypes.c_void_p)
+    a.g_h = gh.ctypes.data_as(ctypes.c_void_p)
+    a.cu_seqlens, a.cu_qtiles, a.cu_ktiles, a.g = _ptr(cud), _ptr(cqd), _ptr(ckd), _ptr(gd)
+    km = None
+    if kv_head_of_q is not None:
+        km = to(kv_head_of_q)
+        a.kv_head_of_q = _ptr(km)
+    a.nseq, a.hq, a.hk, a.d = len(lengths), int(hq), int(hk), int(q.shape[-1])
+    a.causal, a.int8_percent = int(bool(causal)), int(int8_percent)
+    a.masks = _ptr(masks)
+    need = tilemix_route_workspace_size(a)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel()
+    if events is not None:
+        a.event_begin, a.event_end = events[0].cuda_event, events[1].cuda_event
+    tilemix_route_pooled(a, stream)
+    # keep the device metadata alive until the launches have read it
+    masks._route_keepalive = (cud, cqd, ckd, gd, km, workspace)
+    return masks
+
+
 from .prefill import TileMixPrefill  # noqa: E402  (convenience wrapper)
 from .decode import TileMixDecode  # noqa: E402  (convenience wrapper)
 
 __all__ = [
-    "BLOCK_M", "BLOCK_N", "DecodeArgs", "MAX_GROUPS", "PrefillArgs", "TEMPLATES", "TileMixError",
+    "BLOCK_M", "BLOCK_N", "DecodeArgs", "MAX_GROUPS", "PrefillArgs", "RouteArgs", "TEMPLATES",
+    "TileMixError", "route_pooled", "tilemix_route_pooled", "tilemix_route_workspace_size",
     "TileMixDecode", "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
     "tilemix_build_routing", "tilemix_decode_fwd", "tilemix_decode_workspace_size",
     "tilemix_get_error", "tilemix_prefill_fwd",

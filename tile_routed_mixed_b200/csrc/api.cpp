@@ -405,6 +405,101 @@ TILEMIX_API int tilemix_decode_fwd(const tilemix_decode_args* a, void* stream) {
   return TILEMIX_OK;
 }
 
+namespace {
+
+// Host-side validation of pooled-score routing; fills the tile totals.
+int check_route(const tilemix_route_args* a, int* total_qtiles, int* total_ktiles) {
+  if (!a) return TILEMIX_ERR_INVALID_ARG;
+  if (a->d != 64 && a->d != 128) return TILEMIX_ERR_UNSUPPORTED;
+  if (a->nseq < 0 || a->hq < 1 || a->hk < 1 || a->int8_percent < 0 || a->int8_percent > 100 ||
+      (a->causal != 0 && a->causal != 1))
+    return TILEMIX_ERR_INVALID_ARG;
+  if (!a->kv_head_of_q && a->hq % a->hk != 0) return TILEMIX_ERR_INVALID_ARG;
+  if (!a->kv_head_of_q && a->hq / a->hk > 256) return TILEMIX_ERR_UNSUPPORTED;
+  if (a->kv_head_of_q && a->hq > 256) return TILEMIX_ERR_UNSUPPORTED;
+  if (!a->cu_seqlens_h || !a->g_h) return TILEMIX_ERR_INVALID_ARG;
+  if (a->cu_seqlens_h[0] != 0) return TILEMIX_ERR_INVALID_ARG;
+  long long tq = 0, tk = 0;
+  for (int s = 0; s < a->nseq; ++s) {
+    const int L = a->cu_seqlens_h[s + 1] - a->cu_seqlens_h[s];
+    const int g = a->g_h[s];
+    if (L < 0 || g < 1) return TILEMIX_ERR_INVALID_ARG;
+    const int rows = (L + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M;
+    const int kt = (L + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N;
+    // the row with the most legal groups is the last one
+    if (rows > 0 && ((L - 1) / TILEMIX_BLOCK_N) / g + 1 > TILEMIX_MAX_GROUPS)
+      return TILEMIX_ERR_INVALID_ARG;
+    tq += rows;
+    tk += kt;
+  }
+  if (tq > (1LL << 30) || tk > (1LL << 30)) return TILEMIX_ERR_INVALID_ARG;
+  *total_qtiles = static_cast<int>(tq);
+  *total_ktiles = static_cast<int>(tk);
+  if (a->nseq > 0 && tq > 0) {
+    if (!a->q || !a->k || !a->cu_seqlens || !a->cu_qtiles || !a->cu_ktiles || !a->g || !a->masks)
+      return TILEMIX_ERR_INVALID_ARG;
+    if (!aligned16(a->q) || !aligned16(a->k) || (reinterpret_cast<uintptr_t>(a->masks) & 7u))
+      return TILEMIX_ERR_INVALID_ARG;
+  }
+  return TILEMIX_OK;
+}
+
+size_t route_bytes(const tilemix_route_args* a, int tq, int tk, size_t* kbar_off) {
+  *kbar_off = round_up(static_cast<size_t>(tq) * a->hk * a->d * sizeof(float), 256);
+  return round_up(*kbar_off + static_cast<size_t>(tk) * a->hk * a->d * sizeof(float), 256);
+}
+
+}  // namespace
+
+TILEMIX_API int tilemix_route_workspace_size(const tilemix_route_args* a, size_t* bytes) {
+  if (!bytes) return TILEMIX_ERR_INVALID_ARG;
+  int tq = 0, tk = 0;
+  const int rc = check_route(a, &tq, &tk);
+  if (rc != TILEMIX_OK) return rc;
+  size_t off;
+  *bytes = route_bytes(a, tq, tk, &off);
+  return TILEMIX_OK;
+}
+
+TILEMIX_API int tilemix_route_pooled(const tilemix_route_args* a, void* stream) {
+  int tq = 0, tk = 0;
+  int rc = check_route(a, &tq, &tk);
+  if (rc != TILEMIX_OK) return rc;
+  if (a->nseq == 0 || tq == 0) return TILEMIX_OK;
+  size_t kbar_off;
+  const size_t need = route_bytes(a, tq, tk, &kbar_off);
+  if (!a->workspace || a->workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return TILEMIX_ERR_WORKSPACE;
+  tilemix::RouteParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = a->q;
+  p.k = a->k;
+  p.cu_seqlens = a->cu_seqlens;
+  p.cu_qtiles = a->cu_qtiles;
+  p.cu_ktiles = a->cu_ktiles;
+  p.g = a->g;
+  p.kv_head_of_q = a->kv_head_of_q;
+  p.qbar = static_cast<float*>(a->workspace);
+  p.kbar = reinterpret_cast<float*>(static_cast<uint8_t*>(a->workspace) + kbar_off);
+  p.masks = a->masks;
+  p.nseq = a->nseq;
+  p.hq = a->hq;
+  p.hk = a->hk;
+  p.d = a->d;
+  p.causal = a->causal;
+  p.int8_percent = a->int8_percent;
+  p.total_qtiles = tq;
+  p.total_ktiles = tk;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a->event_begin && cudaEventRecord(static_cast<cudaEvent_t>(a->event_begin), st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  if (tilemix::launch_route(p, st) != cudaSuccess) return TILEMIX_ERR_CUDA;
+  if (a->event_end && cudaEventRecord(static_cast<cudaEvent_t>(a->event_end), st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  return TILEMIX_OK;
+}
+
 TILEMIX_API int tilemix_selftest_wait_timeout(int timeout_ms, void* stream) {
   if (timeout_ms < 1 || timeout_ms > 10000) return TILEMIX_ERR_INVALID_ARG;
   if (tilemix::launch_selftest_wait(static_cast<unsigned long long>(timeout_ms) * 1000000ull,

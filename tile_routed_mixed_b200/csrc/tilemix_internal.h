@@ -70,6 +70,22 @@ struct DecodeParams {
   unsigned long long timeout_ns;
 };
 
+// Pooled-score routing (tilemix_route.cu).
+struct RouteParams {
+  const void* q;             // fp16 [T][hq][d]
+  const void* k;             // fp16 [T][hk][d]
+  const int32_t* cu_seqlens;
+  const int32_t* cu_qtiles;
+  const int32_t* cu_ktiles;
+  const int32_t* g;
+  const int32_t* kv_head_of_q;
+  float* qbar;               // workspace: [total_qtiles][hk][d]
+  float* kbar;               // workspace: [total_ktiles][hk][d]
+  uint64_t* masks;           // [total_qtiles][hk]
+  int nseq, hq, hk, d, causal, int8_percent, total_qtiles, total_ktiles;
+};
+int launch_route(const RouteParams& p, cudaStream_t stream);
+
 // Launchers implemented in the CUDA translation unit.  Return cudaError_t.
 int launch_decode(const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_begin,
                   cudaEvent_t ev_end);
