@@ -633,6 +633,139 @@ def run_decode(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------- route path ---
+
+ROUTE_METRIC = "pooled-score adaptive routing tok/s at 4k b8 (3B GQA shape); % of HBM roofline"
+
+
+def run_route(args):
+    """Pooled-score routing words for the whole batch per step.  Its inputs
+    (Q and K, fp16) exceed the 126 MB L2, so no flush."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference" and rank != 0:
+        return
+    w, lengths, g = workload(args.workload, args.template, args.percent)
+    hq, hk, d = w["hq"], w["hk"], w["d"]
+    T = sum(lengths)
+    q, k, _ = synth.make_qkv(rank, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
+    cq, ck = tile_starts(lengths)
+    # algorithmic bytes: Q and K read once, the fp32 means written and read
+    # once, the words written
+    nbytes = (q.nbytes + k.nbytes + 2 * (int(cq[-1]) + int(ck[-1])) * hk * d * 4 +
+              int(cq[-1]) * hk * 8)
+    config = dict(bench_config(args, w, lengths, g), path="route",
+                  l2="no flush: Q and K (%.0f MB per step) exceed the 126 MB L2"
+                     % ((q.nbytes + k.nbytes) / 1e6))
+    sample = lengths[:1]
+    if args.impl == "reference" or not args.no_cpu_baseline:
+        from oracle import adaptive
+        Ts = sample[0]
+        t0 = time.perf_counter()
+        n = 0
+        while n < 1 or time.perf_counter() - t0 < (60.0 if args.impl == "reference" else 10.0):
+            adaptive.route_pooled(q[:Ts], k[:Ts], sample, hq, hk, g[:1], w["causal"],
+                                  w["percent"])
+            n += 1
+        cpu_val = Ts / ((time.perf_counter() - t0) / n)
+        cpu_base = {"value": cpu_val, "unit": "tok/s", "cores": 1, "kind": "oracle",
+                    "sample": "%d runs on the first sequence (%d tokens) of the batch" % (n, Ts)}
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "metric": ROUTE_METRIC, "value": cpu_val,
+                              "unit": "tok/s", "n_gpus": world, "steps": n, "warmup": 0,
+                              "ms_per_step": T / cpu_val * 1e3, "higher_is_better": True,
+                              "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                              "data": "synthetic", "config": config, "cpu_baseline": cpu_base,
+                              "e2e": {"value": cpu_val, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+            return
+    import torch
+    import torch.distributed as dist
+
+    import tile_routed_mixed_b200 as tm
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    qd, kd = torch.from_numpy(q).to(dev), torch.from_numpy(k).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    ws = None
+    for _ in range(args.warmup):
+        m = tm.route_pooled(qd, kd, lengths, hq, hk, g, w["causal"], w["percent"], workspace=ws)
+        ws = m._route_keepalive[-1]
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        b.record(stream)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for e in ev:
+        tm.route_pooled(qd, kd, lengths, hq, hk, g, w["causal"], w["percent"], events=e,
+                        workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    rc = tm.tilemix_get_error(stream)
+    if rc != tm.OK:
+        raise tm.TileMixError(rc, "timed steps")
+    ms = e0.elapsed_time(e1) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    ms, kern_ms = max_over_ranks([ms, kern_ms], device=dev)
+    # end to end: Q and K from pinned host memory in, the words back out
+    qh, kh = torch.from_numpy(q).pin_memory(), torch.from_numpy(k).pin_memory()
+    n_e2e = max(args.steps // 4, 3)
+    words_h = None
+    torch.cuda.synchronize(dev)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(n_e2e):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        m = tm.route_pooled(qd, kd, lengths, hq, hk, g, w["causal"], w["percent"], workspace=ws)
+        words_h = m.to("cpu", non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks([e2.elapsed_time(e3) / n_e2e], device=dev)[0]
+    pk = peaks()
+    tokens = whole_job_tokens(T, world)
+    achieved = nbytes / (kern_ms / 1e3) / 1e9
+    line = {
+        "metric": ROUTE_METRIC, "value": tokens / (ms / 1e3), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"],
+                     "traffic": None, "kernel": "route_pool_kernel x2 + route_words_kernel",
+                     "kernel_ms": kern_ms, "peak_kind": "copy bandwidth (%s)" % pk["source"],
+                     "algorithmic_bytes": nbytes},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tok/s",
+                "h2d_bytes_per_step": int(q.nbytes + k.nbytes),
+                "d2h_bytes_per_step": int(words_h.numel() * 8)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_base
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -643,13 +776,16 @@ def main():
     ap.add_argument("--template", default=None)
     ap.add_argument("--percent", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["prefill", "decode"], default="prefill",
-                    help="prefill (the headline metric) or the decode step with the INT8 K cache")
+    ap.add_argument("--path", choices=["prefill", "decode", "route"], default="prefill",
+                    help="prefill (the headline metric), the decode step with the INT8 K "
+                         "cache, or pooled-score adaptive routing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.path == "decode":
         run_decode(args)
+    elif args.path == "route":
+        run_route(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -15,8 +15,8 @@
 // partial sums added in order; products and sums rounded separately), so the
 // words are reproducible bit for bit.
 //
-//   route_pool_kernel   one CTA per (tile, KV head): 8 x d threads, thread
-//                       (j, c) sums channel c of the items m = j mod 8
+//   route_pool_kernel   one CTA per (tile, KV head): 8 x d/8 threads, thread
+//                       (j, c8) sums channels 8 c8.. of the items m = j mod 8
 //   route_words_kernel  one warp per (query-tile row, KV head)
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -41,13 +41,16 @@ __device__ __forceinline__ int find_seq(const int32_t* cu, int nseq, int x) {
 }
 
 // blockIdx.x: tile (query tiles if kQ, else key tiles), blockIdx.y: KV head.
+// Thread (j, c8): channels [8 c8, 8 c8 + 8) of the items m = j mod 8, read as
+// one 16-byte load per item.
 template <int D, bool kQ>
-__global__ void __launch_bounds__(kRouteLanes * D) route_pool_kernel(RouteParams p) {
+__global__ void __launch_bounds__(kRouteLanes * D / 8) route_pool_kernel(RouteParams p) {
+  constexpr int kC8 = D / 8;  // 16-byte channel chunks per row
   __shared__ float part[kRouteLanes][D];
   __shared__ int heads[256];
   __shared__ int nheads;
   const int tile = blockIdx.x, kv = blockIdx.y;
-  const int c = threadIdx.x % D, j = threadIdx.x / D;
+  const int c8 = threadIdx.x % kC8, j = threadIdx.x / kC8;
   const int32_t* cu_tiles = kQ ? p.cu_qtiles : p.cu_ktiles;
   const int s = find_seq(cu_tiles, p.nseq, tile);
   const int L = __ldg(p.cu_seqlens + s + 1) - __ldg(p.cu_seqlens + s);
@@ -67,29 +70,51 @@ __global__ void __launch_bounds__(kRouteLanes * D) route_pool_kernel(RouteParams
     __syncthreads();
     H = nheads;
   }
-  // items m = head index * R + row (head-major); this thread takes m = j mod 8
-  const int M = H * R;
+  // items m = head index * R + row (head-major); this thread takes m = j mod 8,
+  // i.e. in head hi the rows i = j - hi R (mod 8), ascending: the order of m
   const __half* x = static_cast<const __half*>(kQ ? p.q : p.k);
   const int nh = kQ ? p.hq : p.hk;
-  float acc = 0.f;
-  int hi = j / max(R, 1), i = j - hi * max(R, 1);
-  for (int m = j; m < M; m += kRouteLanes) {
-    const int h = kQ ? heads[hi] : kv;
-    acc = __fadd_rn(acc, __half2float(x[(static_cast<size_t>(row0 + i) * nh + h) * D + c]));
-    i += kRouteLanes;
-    while (i >= R) {
-      i -= R;
-      ++hi;
+  const size_t step = static_cast<size_t>(kRouteLanes) * nh * D;  // elements between items
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  auto add8 = [&](const uint4& u) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
+      acc[2 * e] = __fadd_rn(acc[2 * e], f.x);
+      acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], f.y);
     }
+  };
+  for (int hi = 0; hi < H; ++hi) {
+    const int h = kQ ? heads[hi] : kv;
+    int i = (j - hi * R) % kRouteLanes;
+    if (i < 0) i += kRouteLanes;
+    const __half* ptr = x + (static_cast<size_t>(row0 + i) * nh + h) * D + 8 * c8;
+    // loads issued four ahead; the adds stay in ascending row order
+    for (; i + 3 * kRouteLanes < R; i += 4 * kRouteLanes, ptr += 4 * step) {
+      const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(ptr));
+      const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(ptr + step));
+      const uint4 u2 = __ldg(reinterpret_cast<const uint4*>(ptr + 2 * step));
+      const uint4 u3 = __ldg(reinterpret_cast<const uint4*>(ptr + 3 * step));
+      add8(u0);
+      add8(u1);
+      add8(u2);
+      add8(u3);
+    }
+    for (; i < R; i += kRouteLanes, ptr += step) add8(__ldg(reinterpret_cast<const uint4*>(ptr)));
   }
-  part[j][c] = acc;
+  const int M = H * R;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[j][8 * c8 + e] = acc[e];
   __syncthreads();
-  if (j == 0) {
+  float* out = kQ ? p.qbar : p.kbar;
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
     float tot = part[0][c];
 #pragma unroll
     for (int q = 1; q < kRouteLanes; ++q) tot = __fadd_rn(tot, part[q][c]);
     if (M > 0) tot = __fdiv_rn(tot, static_cast<float>(M));
-    float* out = kQ ? p.qbar : p.kbar;
     out[(static_cast<size_t>(tile) * p.hk + kv) * D + c] = tot;
   }
 }
@@ -144,8 +169,15 @@ __global__ void __launch_bounds__(128) route_words_kernel(RouteParams p) {
     for (int kt = b * gs; kt < min((b + 1) * gs, lt + 1); ++kt) {
       const float* kb = p.kbar + (static_cast<size_t>(ck + kt) * p.hk + kv) * D;
       float dot = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) dot = __fadd_rn(dot, __fmul_rn(__ldg(qb + c), __ldg(kb + c)));
+#pragma unroll 4
+      for (int c = 0; c < D; c += 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(qb + c));
+        const float4 b4 = __ldg(reinterpret_cast<const float4*>(kb + c));
+        dot = __fadd_rn(dot, __fmul_rn(a.x, b4.x));
+        dot = __fadd_rn(dot, __fmul_rn(a.y, b4.y));
+        dot = __fadd_rn(dot, __fmul_rn(a.z, b4.z));
+        dot = __fadd_rn(dot, __fmul_rn(a.w, b4.w));
+      }
       best = fmaxf(best, dot);
     }
     sc[h] = best;
@@ -171,12 +203,12 @@ template <int D>
 cudaError_t launch_route_d(const RouteParams& p, cudaStream_t stream) {
   if (p.total_qtiles > 0)
     route_pool_kernel<D, true>
-        <<<dim3(p.total_qtiles, p.hk), kRouteLanes * D, 0, stream>>>(p);
+        <<<dim3(p.total_qtiles, p.hk), kRouteLanes * D / 8, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (p.total_ktiles > 0)
     route_pool_kernel<D, false>
-        <<<dim3(p.total_ktiles, p.hk), kRouteLanes * D, 0, stream>>>(p);
+        <<<dim3(p.total_ktiles, p.hk), kRouteLanes * D / 8, 0, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long warps = static_cast<long long>(p.total_qtiles) * p.hk;
   if (warps > 0)
