@@ -643,3 +643,91 @@ def test_adaptive_pooled_means_by_brute_force():
     # key tile 3 is the 64 rows of sequence 1
     np.testing.assert_allclose(kb[3, 0], k[130:194, 0].astype(np.float64).mean(axis=0),
                                rtol=1e-5, atol=1e-6)
+
+
+# ------------------------------------------------------- importance-mass probe --
+from oracle import mass as om  # noqa: E402
+
+
+def _words_all(lengths, hk, bit):
+    n = sum(oracle.n_qtiles(L) for L in lengths)
+    return np.full((n, hk), np.uint64((1 << 64) - 1 if bit else 0), dtype=np.uint64)
+
+
+def test_mass_probe_all_fp16_and_all_int8_words():
+    rng = np.random.default_rng(11)
+    lengths, hq, hk, d = [200, 70], 2, 1, 64
+    q = rng.standard_normal((270, hq, d)).astype(np.float16)
+    k = rng.standard_normal((270, hk, d)).astype(np.float16)
+    r0 = om.probe_rows(q, k, _words_all(lengths, hk, 0), [1, 1], lengths, True)
+    assert np.all(r0["m8"] == 0) and np.all(r0["h8"] == 0)
+    r1 = om.probe_rows(q, k, _words_all(lengths, hk, 1), [1, 1], lengths, True)
+    np.testing.assert_allclose(r1["m8"], 1.0, atol=1e-12)
+    np.testing.assert_allclose(r1["h8"], r1["h"], atol=1e-12)
+    assert np.all(r1["h"] <= 1 + 1e-12) and np.all(r1["h"] > 0)
+
+
+def test_mass_probe_uniform_scores_closed_form():
+    # q = 0: every legal key scores 0, P is uniform over the i + 1 legal keys,
+    # every key is high-importance, and the INT8 mass is the INT8 key count
+    # over i + 1
+    lengths, hq, hk, d = [300], 1, 1, 64
+    q = np.zeros((300, hq, d), dtype=np.float16)
+    k = np.random.default_rng(1).standard_normal((300, hk, d)).astype(np.float16)
+    words = np.array([[0b101], [0b1010], [0b10001]], dtype=np.uint64)  # one word per 128 rows
+    r = om.probe_rows(q, k, words, [1], lengths, True)
+    for i in range(300):
+        w = int(words[i // 128, 0])
+        n8 = sum(1 for j in range(i + 1) if (w >> (j // 64)) & 1)
+        assert abs(r["m8"][0, i] - n8 / (i + 1)) < 1e-12
+        assert abs(r["h"][0, i] - 1.0) < 1e-12
+        assert abs(r["h8"][0, i] - n8 / (i + 1)) < 1e-12
+
+
+def test_mass_probe_two_key_hand_case():
+    # row 1 sees keys 0 and 1 with scores 0 and a: P = (1, e^a) / (1 + e^a);
+    # with a = 4 ln 2 + 0.1 key 0 falls below the 2^-4 threshold (delta 4)
+    d = 64
+    a = 4 * math.log(2) + 0.1
+    q = np.zeros((2, 1, d), dtype=np.float16)
+    k = np.zeros((2, 1, d), dtype=np.float16)
+    q[1, 0, 0] = np.float16(1.0)
+    k[1, 0, 0] = np.float16(a * math.sqrt(d))
+    k_eff = float(np.float16(a * math.sqrt(d))) / math.sqrt(d)      # the fp16-rounded score
+    words = np.array([[0b1]], dtype=np.uint64)                       # tile 0 (both keys) INT8
+    r = om.probe_rows(q, k, words, [1], [2], True)
+    p1 = math.exp(k_eff) / (1 + math.exp(k_eff))
+    assert k_eff > 4 * math.log(2)
+    assert abs(r["m8"][0, 1] - 1.0) < 1e-12
+    assert abs(r["h"][0, 1] - p1) < 1e-12
+    assert abs(r["h8"][0, 1] - p1) < 1e-12
+    assert abs(om.exposure(r["h"], r["h8"]) - 1.0) < 1e-12
+
+
+def test_mass_probe_matches_python_loops():
+    rng = np.random.default_rng(5)
+    lengths, hq, hk, d = [150, 9], 2, 1, 64
+    T = sum(lengths)
+    q = (rng.standard_normal((T, hq, d)) * 0.5).astype(np.float16)
+    k = rng.standard_normal((T, hk, d)).astype(np.float16)
+    words = np.array([[0b01], [0b10], [0b1]], dtype=np.uint64)
+    r = om.probe_rows(q, k, words, [1, 1], lengths, True, delta=2.0)
+    start, cq = 0, 0
+    for s, L in enumerate(lengths):
+        for h in range(hq):
+            for i in range(0, L, 7):
+                sc = [sum(float(q[start + i, h, c]) * float(k[start + j, 0, c]) for c in range(d))
+                      / 8.0 for j in range(i + 1)]
+                mx = max(sc)
+                e = [math.exp(x - mx) for x in sc]
+                tot = sum(e)
+                w = int(words[cq + i // 128, 0])
+                m8 = sum(e[j] for j in range(i + 1) if (w >> (j // 64)) & 1) / tot
+                hh = sum(e[j] for j in range(i + 1) if sc[j] >= mx - 2 * math.log(2)) / tot
+                h8 = sum(e[j] for j in range(i + 1)
+                         if sc[j] >= mx - 2 * math.log(2) and (w >> (j // 64)) & 1) / tot
+                assert abs(r["m8"][h, start + i] - m8) < 1e-10
+                assert abs(r["h"][h, start + i] - hh) < 1e-10
+                assert abs(r["h8"][h, start + i] - h8) < 1e-10
+        start += L
+        cq += oracle.n_qtiles(L)
