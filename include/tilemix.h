@@ -342,6 +342,52 @@ int tilemix_route_workspace_size(const tilemix_route_args* args, size_t* bytes);
  * if a launch fails.  All argument errors are returned before any launch. */
 int tilemix_route_pooled(const tilemix_route_args* args, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Importance-mass exposure probe.
+ *
+ * The pages report that static SpTrans routing at 25% INT8 coverage sends only
+ * about 8.5% of the selected high-importance attention mass to INT8
+ * ("Precision Has a Map: TileMix Routes INT8 Inside Dense Attention",
+ * cognaptus.com, last section; agihunt.info summary, results paragraph), and do
+ * not say how interactions are selected.  Reading: P_ij is row i's softmax
+ * over its legal keys of the full-precision scores (fp16 inputs, fp32
+ * scores), and the high-importance keys are those with
+ * P_ij >= 2^-delta_log2 * max_j P_ij.  Per (query head, token) the probe
+ * writes
+ *   m8 = sum of P_ij over INT8-routed legal keys,
+ *   h  = sum of P_ij over the high-importance keys,
+ *   h8 = sum of P_ij over the high-importance INT8-routed keys,
+ * where a key is INT8-routed when the row's routing word (the same words the
+ * attention path reads) has its group's bit set.  A batch's exposure is
+ * sum h8 / sum h.  One launch; nothing is allocated. */
+typedef struct tilemix_mass_args {
+  const void* q;              /* device fp16 [T][hq][d], 16-B aligned */
+  const void* k;              /* device fp16 [T][hk][d], 16-B aligned */
+  const int32_t* cu_seqlens_h;/* host [nseq + 1]: validation and grid size */
+  const int32_t* g_h;         /* host [nseq] */
+  const int32_t* cu_seqlens;  /* device copies of the same values ... */
+  const int32_t* cu_qtiles;   /* ... and the tile offsets (tilemix_tile_offsets) */
+  const int32_t* cu_ktiles;
+  const int32_t* g;
+  const uint64_t* masks;      /* device [total_qtiles][hk] routing words */
+  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk) */
+  int nseq, hq, hk, d;        /* d in {64, 128} */
+  int causal;                 /* 0 or 1 */
+  float softmax_scale;        /* 0 => 1 / sqrt(d) */
+  float delta_log2;           /* > 0; 4 => keys within a factor 16 of the row's largest P */
+  float* m8;                  /* device out [hq][T] */
+  float* h;                   /* device out [hq][T] */
+  float* h8;                  /* device out [hq][T] */
+  void* event_begin;          /* NULL, or cudaEvent_t recorded around the launch */
+  void* event_end;
+} tilemix_mass_args;
+
+/* The probe as described above.  INVALID_ARG on a NULL required pointer, a
+ * misaligned tensor, delta_log2 <= 0, a bad causal flag, g or lengths, or
+ * hq % hk != 0 without a head map; UNSUPPORTED for d not in {64, 128}; CUDA if
+ * the launch fails.  Argument errors return before any launch. */
+int tilemix_mass_probe(const tilemix_mass_args* args, void* stream);
+
 /* Self test of the failure path: enqueues one warp that waits on a device
  * barrier nothing ever signals, with the same bounded wait the attention
  * kernel uses, limited to timeout_ms (1..10000).  The wait gives up, latches

@@ -234,3 +234,47 @@ def test_route_argument_checks_are_synchronous():
     a = _fake_route(empty, np.zeros(0, np.int32), q=None, k=None)
     a.nseq = 0
     assert L.tilemix_route_pooled(ctypes.byref(a), None) == tm.OK
+
+
+def test_mass_probe_argument_checks_are_synchronous():
+    L = ctypes.CDLL(tm.LIB_PATH)
+    L.tilemix_mass_probe.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    cu = np.array([0, 300, 1300], dtype=np.int32)
+    g = np.array([1, 1], dtype=np.int32)
+
+    def fake(**over):
+        a = tm.MassArgs()
+        for f in ("q", "k", "cu_seqlens", "cu_qtiles", "cu_ktiles", "g", "masks", "m8", "h", "h8"):
+            setattr(a, f, 4096)
+        a.cu_seqlens_h = cu.ctypes.data_as(ctypes.c_void_p)
+        a.g_h = g.ctypes.data_as(ctypes.c_void_p)
+        a.nseq, a.hq, a.hk, a.d, a.causal, a.delta_log2 = 2, 6, 2, 128, 1, 4.0
+        for k, v in over.items():
+            setattr(a, k, v)
+        return a
+
+    cases = [
+        (dict(d=96), tm.ERR_UNSUPPORTED),
+        (dict(delta_log2=0.0), tm.ERR_INVALID_ARG),
+        (dict(delta_log2=float("inf")), tm.ERR_INVALID_ARG),
+        (dict(delta_log2=float("nan")), tm.ERR_INVALID_ARG),
+        (dict(softmax_scale=-1.0), tm.ERR_INVALID_ARG),
+        (dict(causal=3), tm.ERR_INVALID_ARG),
+        (dict(hq=5, hk=2), tm.ERR_INVALID_ARG),
+        (dict(h8=None), tm.ERR_INVALID_ARG),
+        (dict(q=4104), tm.ERR_INVALID_ARG),
+        (dict(g_h=None), tm.ERR_INVALID_ARG),
+    ]
+    for over, want in cases:
+        assert L.tilemix_mass_probe(ctypes.byref(fake(**over)), None) == want, over
+    long_seq = np.array([0, 64 * 64 + 1], dtype=np.int32)
+    one = np.array([1], dtype=np.int32)
+    a = fake(nseq=1)
+    a.cu_seqlens_h = long_seq.ctypes.data_as(ctypes.c_void_p)
+    a.g_h = one.ctypes.data_as(ctypes.c_void_p)
+    assert L.tilemix_mass_probe(ctypes.byref(a), None) == tm.ERR_INVALID_ARG   # 65 groups
+    empty = np.array([0, 0], dtype=np.int32)
+    a = fake(nseq=1, q=None, k=None)
+    a.cu_seqlens_h = empty.ctypes.data_as(ctypes.c_void_p)
+    a.g_h = one.ctypes.data_as(ctypes.c_void_p)
+    assert L.tilemix_mass_probe(ctypes.byref(a), None) == tm.OK                # nothing to do

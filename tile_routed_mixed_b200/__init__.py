@@ -84,6 +84,22 @@ class RouteArgs(ctypes.Structure):
     ]
 
 
+class MassArgs(ctypes.Structure):
+    """Mirror of ``tilemix_mass_args``."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
+        ("cu_seqlens_h", ctypes.c_void_p), ("g_h", ctypes.c_void_p),
+        ("cu_seqlens", ctypes.c_void_p), ("cu_qtiles", ctypes.c_void_p),
+        ("cu_ktiles", ctypes.c_void_p), ("g", ctypes.c_void_p), ("masks", ctypes.c_void_p),
+        ("kv_head_of_q", ctypes.c_void_p),
+        ("nseq", ctypes.c_int), ("hq", ctypes.c_int), ("hk", ctypes.c_int), ("d", ctypes.c_int),
+        ("causal", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+        ("delta_log2", ctypes.c_float),
+        ("m8", ctypes.c_void_p), ("h", ctypes.c_void_p), ("h8", ctypes.c_void_p),
+        ("event_begin", ctypes.c_void_p), ("event_end", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -124,6 +140,8 @@ def lib():
                                                    ctypes.POINTER(ctypes.c_size_t)]
         L.tilemix_route_pooled.restype = I
         L.tilemix_route_pooled.argtypes = [ctypes.POINTER(RouteArgs), P]
+        L.tilemix_mass_probe.restype = I
+        L.tilemix_mass_probe.argtypes = [ctypes.POINTER(MassArgs), P]
         L.tilemix_selftest_wait_timeout.restype = I
         L.tilemix_selftest_wait_timeout.argtypes = [I, P]
         L.tilemix_get_error.restype = I
@@ -337,12 +355,55 @@ def route_pooled(q, k, lengths, hq, hk, g, causal, int8_percent, kv_head_of_q=No
     return masks
 
 
+def tilemix_mass_probe(args: MassArgs, stream=None):
+    _check(lib().tilemix_mass_probe(ctypes.byref(args), _stream_handle(stream)),
+           "tilemix_mass_probe")
+
+
+def mass_probe(q, k, masks, lengths, hq, hk, g, causal=True, delta_log2=4.0, kv_head_of_q=None,
+               softmax_scale=0.0, stream=None, events=None):
+    """Per (query head, token) m8, h, h8 (fp32 tensors [hq, T]) on q's device."""
+    import numpy as np
+    import torch
+    dev = q.device
+    lengths = [int(x) for x in lengths]
+    cu = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lengths)
+    cq, ck = tilemix_tile_offsets(cu)
+    gh = np.ascontiguousarray(np.asarray(g, dtype=np.int32))
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    cud, cqd, ckd, gd = to(cu), to(cq), to(ck), to(gh)
+    if isinstance(masks, np.ndarray):
+        masks = torch.from_numpy(np.ascontiguousarray(masks, dtype=np.uint64).view(np.int64)).to(dev)
+    T = int(cu[-1])
+    out = [torch.empty((int(hq), T), dtype=torch.float32, device=dev) for _ in range(3)]
+    a = MassArgs()
+    a.q, a.k = _ptr(q), _ptr(k)
+    a.cu_seqlens_h = cu.ctypes.data_as(ctypes.c_void_p)
+    a.g_h = gh.ctypes.data_as(ctypes.c_void_p)
+    a.cu_seqlens, a.cu_qtiles, a.cu_ktiles, a.g = _ptr(cud), _ptr(cqd), _ptr(ckd), _ptr(gd)
+    a.masks = _ptr(masks)
+    km = None
+    if kv_head_of_q is not None:
+        km = to(kv_head_of_q)
+        a.kv_head_of_q = _ptr(km)
+    a.nseq, a.hq, a.hk, a.d = len(lengths), int(hq), int(hk), int(q.shape[-1])
+    a.causal, a.softmax_scale, a.delta_log2 = int(bool(causal)), float(softmax_scale), float(delta_log2)
+    a.m8, a.h, a.h8 = _ptr(out[0]), _ptr(out[1]), _ptr(out[2])
+    if events is not None:
+        a.event_begin, a.event_end = events[0].cuda_event, events[1].cuda_event
+    tilemix_mass_probe(a, stream)
+    out[0]._mass_keepalive = (cud, cqd, ckd, gd, km, masks)
+    return tuple(out)
+
+
 from .prefill import TileMixPrefill  # noqa: E402  (convenience wrapper)
 from .decode import TileMixDecode  # noqa: E402  (convenience wrapper)
 
 __all__ = [
     "BLOCK_M", "BLOCK_N", "DecodeArgs", "MAX_GROUPS", "PrefillArgs", "RouteArgs", "TEMPLATES",
     "TileMixError", "route_pooled", "tilemix_route_pooled", "tilemix_route_workspace_size",
+    "MassArgs", "mass_probe", "tilemix_mass_probe",
     "TileMixDecode", "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
     "tilemix_build_routing", "tilemix_decode_fwd", "tilemix_decode_workspace_size",
     "tilemix_get_error", "tilemix_prefill_fwd",

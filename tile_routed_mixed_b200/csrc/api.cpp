@@ -500,6 +500,62 @@ TILEMIX_API int tilemix_route_pooled(const tilemix_route_args* a, void* stream) 
   return TILEMIX_OK;
 }
 
+TILEMIX_API int tilemix_mass_probe(const tilemix_mass_args* a, void* stream) {
+  if (!a) return TILEMIX_ERR_INVALID_ARG;
+  if (a->d != 64 && a->d != 128) return TILEMIX_ERR_UNSUPPORTED;
+  if (a->nseq < 0 || a->hq < 1 || a->hk < 1 || (a->causal != 0 && a->causal != 1) ||
+      !(a->delta_log2 > 0.f) || std::isinf(a->delta_log2) || !(a->softmax_scale >= 0.f) ||
+      std::isinf(a->softmax_scale))
+    return TILEMIX_ERR_INVALID_ARG;
+  if (!a->kv_head_of_q && a->hq % a->hk != 0) return TILEMIX_ERR_INVALID_ARG;
+  if (!a->cu_seqlens_h || !a->g_h || a->cu_seqlens_h[0] != 0) return TILEMIX_ERR_INVALID_ARG;
+  long long blocks = 0;
+  for (int s = 0; s < a->nseq; ++s) {
+    const int L = a->cu_seqlens_h[s + 1] - a->cu_seqlens_h[s];
+    if (L < 0 || a->g_h[s] < 1) return TILEMIX_ERR_INVALID_ARG;
+    if (L > 0 && ((L - 1) / TILEMIX_BLOCK_N) / a->g_h[s] + 1 > TILEMIX_MAX_GROUPS)
+      return TILEMIX_ERR_INVALID_ARG;
+    blocks += (L + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N;
+  }
+  const long long T = a->nseq > 0 ? a->cu_seqlens_h[a->nseq] : 0;
+  if (blocks > (1LL << 30) || T > (1LL << 31) - 1) return TILEMIX_ERR_INVALID_ARG;
+  if (blocks == 0) return TILEMIX_OK;
+  if (!a->q || !a->k || !a->cu_seqlens || !a->cu_qtiles || !a->cu_ktiles || !a->g ||
+      !a->masks || !a->m8 || !a->h || !a->h8)
+    return TILEMIX_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k)) return TILEMIX_ERR_INVALID_ARG;
+  tilemix::MassParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = a->q;
+  p.k = a->k;
+  p.cu_seqlens = a->cu_seqlens;
+  p.cu_qtiles = a->cu_qtiles;
+  p.cu_ktiles = a->cu_ktiles;
+  p.masks = a->masks;
+  p.g = a->g;
+  p.kv_head_of_q = a->kv_head_of_q;
+  p.m8 = a->m8;
+  p.h = a->h;
+  p.h8 = a->h8;
+  p.nseq = a->nseq;
+  p.hq = a->hq;
+  p.hk = a->hk;
+  p.d = a->d;
+  p.causal = a->causal;
+  p.total_blocks = static_cast<int>(blocks);
+  p.total_tokens = static_cast<int>(T);
+  const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(a->d));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.delta_log2 = a->delta_log2;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a->event_begin && cudaEventRecord(static_cast<cudaEvent_t>(a->event_begin), st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  if (tilemix::launch_mass_probe(p, st) != cudaSuccess) return TILEMIX_ERR_CUDA;
+  if (a->event_end && cudaEventRecord(static_cast<cudaEvent_t>(a->event_end), st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  return TILEMIX_OK;
+}
+
 TILEMIX_API int tilemix_selftest_wait_timeout(int timeout_ms, void* stream) {
   if (timeout_ms < 1 || timeout_ms > 10000) return TILEMIX_ERR_INVALID_ARG;
   if (tilemix::launch_selftest_wait(static_cast<unsigned long long>(timeout_ms) * 1000000ull,

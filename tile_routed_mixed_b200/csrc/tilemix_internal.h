@@ -86,6 +86,24 @@ struct RouteParams {
 };
 int launch_route(const RouteParams& p, cudaStream_t stream);
 
+// Importance-mass exposure probe (tilemix_mass.cu).
+struct MassParams {
+  const void* q;             // fp16 [T][hq][d]
+  const void* k;             // fp16 [T][hk][d]
+  const int32_t* cu_seqlens;
+  const int32_t* cu_qtiles;
+  const int32_t* cu_ktiles;  // also the offsets of the 64-row query blocks
+  const uint64_t* masks;     // [total_qtiles][hk]
+  const int32_t* g;
+  const int32_t* kv_head_of_q;
+  float* m8;                 // [hq][T]
+  float* h;                  // [hq][T]
+  float* h8;                 // [hq][T]
+  int nseq, hq, hk, d, causal, total_blocks, total_tokens;
+  float scale_log2, delta_log2;
+};
+int launch_mass_probe(const MassParams& p, cudaStream_t stream);
+
 // Launchers implemented in the CUDA translation unit.  Return cudaError_t.
 int launch_decode(const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_begin,
                   cudaEvent_t ev_end);
