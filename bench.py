@@ -766,6 +766,166 @@ def run_route(args):
         dist.destroy_process_group()
 
 
+# -------------------------------------------------------------- mass path ---
+
+MASS_METRIC = "importance-mass exposure probe tok/s at 4k b8 (3B GQA shape); % of FP16 tensor peak"
+
+
+def mass_flops(lengths, hq, d, causal):
+    """Score FLOPs of the probe: two sweeps over each 64-row block's legal key tiles."""
+    f = 0
+    for L in lengths:
+        for b in range((L + 63) // 64):
+            last = ((min(64 * b + 64, L) - 1) // 64) if causal else (L - 1) // 64
+            f += (last + 1) * 64 * 64 * 2 * d
+    return 2 * f * hq
+
+
+def run_mass(args):
+    """The probe over the whole batch per step (the bench's routing words),
+    plus the batch exposure for several routings (computed once, untimed)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference" and rank != 0:
+        return
+    w, lengths, g = workload(args.workload, args.template, args.percent)
+    hq, hk, d, causal = w["hq"], w["hk"], w["d"], w["causal"]
+    T = sum(lengths)
+    q, k, _ = synth.make_qkv(rank, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
+    config = dict(bench_config(args, w, lengths, g), path="mass", delta_log2=4.0,
+                  l2="no flush: Q and K (%.0f MB per step) exceed the 126 MB L2"
+                     % ((q.nbytes + k.nbytes) / 1e6))
+    flops = mass_flops(lengths, hq, d, causal)
+    cpu_base = None
+    if args.impl == "reference" or not args.no_cpu_baseline:
+        import oracle
+        from oracle import mass as om
+        Ls = min(lengths[0], 1024)
+        sm, _, _ = oracle.build_routing(w["template"], w["percent"], w["routing_seed"], [Ls], hk,
+                                        g[:1], causal)
+        t0 = time.perf_counter()
+        n = 0
+        while n < 1 or time.perf_counter() - t0 < 10.0:
+            om.probe_rows(q[:Ls], k[:Ls], sm, g[:1], [Ls], causal)
+            n += 1
+        dt = (time.perf_counter() - t0) / n
+        # tokens/s scaled by the causal work: a 4096-row sequence costs 16x a 1024-row one
+        scale = sum((L / Ls) ** 2 for L in lengths)
+        cpu_val = T / (dt * scale)
+        cpu_base = {"value": cpu_val, "unit": "tok/s", "cores": host_cores(), "kind": "oracle",
+                    "sample": "%d runs on the first %d tokens of sequence 0, scaled by the batch's "
+                              "quadratic work" % (n, Ls)}
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "metric": MASS_METRIC, "value": cpu_val,
+                              "unit": "tok/s", "n_gpus": world, "steps": n, "warmup": 0,
+                              "ms_per_step": T / cpu_val * 1e3, "higher_is_better": True,
+                              "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                              "data": "synthetic", "config": config, "cpu_baseline": cpu_base,
+                              "e2e": {"value": cpu_val, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+            return
+    import torch
+    import torch.distributed as dist
+
+    import tile_routed_mixed_b200 as tm
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    cu = synth.cu_seqlens_of(lengths)
+    masks, _, _ = tm.tilemix_build_routing(w["template"], w["percent"], w["routing_seed"], cu, hk,
+                                           g, causal)
+    qd, kd = torch.from_numpy(q).to(dev), torch.from_numpy(k).to(dev)
+    md = torch.from_numpy(np.ascontiguousarray(masks).view(np.int64)).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        tm.mass_probe(qd, kd, md, lengths, hq, hk, g, causal)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        b.record(stream)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for e in ev:
+        tm.mass_probe(qd, kd, md, lengths, hq, hk, g, causal, events=e)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    rc = tm.tilemix_get_error(stream)
+    if rc != tm.OK:
+        raise tm.TileMixError(rc, "timed steps")
+    ms = e0.elapsed_time(e1) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    ms, kern_ms = max_over_ranks([ms, kern_ms], device=dev)
+    # end to end: Q and K from pinned host memory in, the three row arrays out
+    qh, kh = torch.from_numpy(q).pin_memory(), torch.from_numpy(k).pin_memory()
+    n_e2e = max(args.steps // 4, 3)
+    torch.cuda.synchronize(dev)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    out_bytes = 0
+    for _ in range(n_e2e):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        outs = tm.mass_probe(qd, kd, md, lengths, hq, hk, g, causal)
+        hosts = [x.to("cpu", non_blocking=True) for x in outs]
+        out_bytes = sum(x.numel() * 4 for x in hosts)
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks([e2.elapsed_time(e3) / n_e2e], device=dev)[0]
+    # exposure of several routings of this batch (untimed)
+    expo = {}
+    for tpl, pct in (("sptrans", 25), ("sptrans", 50), ("sptrans", 75), ("adaptive", 25),
+                     ("adaptive", 75)):
+        if tpl == "adaptive":
+            mw = tm.route_pooled(qd, kd, lengths, hq, hk, g, causal, pct)
+        else:
+            mm, _, _ = tm.tilemix_build_routing(tpl, pct, w["routing_seed"], cu, hk, g, causal)
+            mw = torch.from_numpy(np.ascontiguousarray(mm).view(np.int64)).to(dev)
+        m8, hh, h8 = tm.mass_probe(qd, kd, mw, lengths, hq, hk, g, causal)
+        expo["%s%d" % (tpl, pct)] = {
+            "int8_share_of_high_importance_mass": float(h8.double().sum() / hh.double().sum()),
+            "int8_share_of_all_mass": float(m8.double().mean())}
+    pk = peaks()
+    tokens = whole_job_tokens(T, world)
+    achieved = flops / (kern_ms / 1e3) / 1e12
+    line = {
+        "metric": MASS_METRIC, "value": tokens / (ms / 1e3), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": config,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                     "kernel": "mass_probe_kernel<128>", "kernel_ms": kern_ms,
+                     "peak_kind": "dense bf16 burst (%s), fp16 taken at the same rate" % pk["source"],
+                     "score_flops": flops},
+        "exposure": expo,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tok/s",
+                "h2d_bytes_per_step": int(q.nbytes + k.nbytes), "d2h_bytes_per_step": int(out_bytes)},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and cpu_base is not None:
+        line["cpu_baseline"] = cpu_base
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -776,7 +936,7 @@ def main():
     ap.add_argument("--template", default=None)
     ap.add_argument("--percent", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["prefill", "decode", "route"], default="prefill",
+    ap.add_argument("--path", choices=["prefill", "decode", "route", "mass"], default="prefill",
                     help="prefill (the headline metric), the decode step with the INT8 K "
                          "cache, or pooled-score adaptive routing")
     args = ap.parse_args()
@@ -786,6 +946,8 @@ def main():
         run_decode(args)
     elif args.path == "route":
         run_route(args)
+    elif args.path == "mass":
+        run_mass(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
