@@ -11,7 +11,9 @@ own splitmix64), and plain C in fp64 / int64 for the attention rows
 (``attention_oracle.c``, OpenMP over rows, no blocking); the decode step
 (``decode.py``) composes those; ``adaptive.py`` restates the pooled-score
 (content-aware) routing policy in fp32 in its stated order; ``mass.py`` is the
-fp64 importance-mass exposure probe.  It shares no code,
+fp64 importance-mass exposure probe; ``fp8.py`` the e4m3 codec and block
+quantiser of the FP8 low path (the C attention oracle reads those codes when
+asked to).  It shares no code,
 header, table or constant generator with the CUDA path.
 
 Pages followed: "TileMix: Tile-Centric Mixed-Precision Attention for LLM
@@ -26,7 +28,7 @@ brute force, closed forms, hand-derived words and invariants the pages fix.
 The fp16 output values themselves have no printed worked example on the pages:
 beyond those invariants, output-value parity is unpinned.
 """
-from . import adaptive, mass
+from . import adaptive, fp8, mass
 from .attention import all_rows, attention_rows, build, half_to_double, int_scores
 from .decode import decode_rows, quantize_rows
 from .quant import quantize_blocks, quantize_k, quantize_q
@@ -35,7 +37,7 @@ from .routing import (BLOCK_M, BLOCK_N, MAX_GROUPS, TEMPLATES, auto_g, build_rou
                       n_qtiles, tile_offsets)
 
 __all__ = [
-    "adaptive", "mass", "BLOCK_M", "BLOCK_N", "MAX_GROUPS", "TEMPLATES", "all_rows", "attention_rows", "auto_g",
+    "adaptive", "fp8", "mass", "BLOCK_M", "BLOCK_N", "MAX_GROUPS", "TEMPLATES", "all_rows", "attention_rows", "auto_g",
     "build", "build_routing", "decode_rows", "fp16_groups", "half_to_double", "int8_target",
     "int_scores",
     "last_legal_tile", "legal_groups", "n_ktiles", "n_qtiles", "quantize_blocks",

@@ -37,6 +37,8 @@ def _load():
         lib.oracle_attention_rows.restype = I
         lib.oracle_attention_rows.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I,
                                               I, I, P, ctypes.c_double, P, ctypes.c_int64, P, P]
+        lib.oracle_attention_rows_fmt.restype = I
+        lib.oracle_attention_rows_fmt.argtypes = lib.oracle_attention_rows.argtypes + [I]
         lib.oracle_int_scores.restype = I
         lib.oracle_int_scores.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P]
         lib.oracle_half_to_double.restype = ctypes.c_double
@@ -60,10 +62,11 @@ def all_rows(lengths, hq):
 
 
 def attention_rows(q, k, v, q8, q_scale, k8, k_scale, masks, g, lengths, causal,
-                   kv_map=None, scale=None, rows=None):
+                   kv_map=None, scale=None, rows=None, low="int8"):
     """fp64 output rows and LSE of tile-routed attention.
 
-    q [T,hq,d], k/v [T,hk,d] float16; q8/k8 int8 codes in the same layouts;
+    q [T,hq,d], k/v [T,hk,d] float16; q8/k8 the low-precision codes in the
+    same layouts (int8, or e4m3 bytes when low == "fp8");
     q_scale [hq, total_qtiles], k_scale [hk, total_ktiles] float32;
     masks [total_qtiles, hk] uint64; g one grouping factor per sequence;
     rows: [n, 3] (sequence, head, row) or None for every row.
@@ -85,15 +88,18 @@ def attention_rows(q, k, v, q8, q_scale, k8, k_scale, masks, g, lengths, causal,
     n = rows.shape[0]
     out = np.zeros((n, d), dtype=np.float64)
     lse = np.zeros(n, dtype=np.float64)
+    if low not in ("int8", "fp8"):
+        raise ValueError(low)
     args = [_c(q, np.float16).view(np.uint16), _c(k, np.float16).view(np.uint16),
-            _c(v, np.float16).view(np.uint16), _c(q8, np.int8), _c(q_scale, np.float32),
-            _c(k8, np.int8), _c(k_scale, np.float32), _c(masks, np.uint64),
+            _c(v, np.float16).view(np.uint16), _c(q8, q8.dtype).view(np.int8),
+            _c(q_scale, np.float32), _c(k8, k8.dtype).view(np.int8), _c(k_scale, np.float32),
+            _c(masks, np.uint64),
             _c(g, np.int32), cu, cu_q, cu_k]
     keep = args + [_c(kv_map, np.int32), rows, out, lse]
-    rc = lib.oracle_attention_rows(
+    rc = lib.oracle_attention_rows_fmt(
         *[a.ctypes.data for a in args], len(lengths), int(cu_q[-1]), int(cu_k[-1]), hq, hk, d,
         int(bool(causal)), keep[12].ctypes.data, float(scale), rows.ctypes.data, n,
-        out.ctypes.data, lse.ctypes.data)
+        out.ctypes.data, lse.ctypes.data, int(low == "fp8"))
     if rc != 0:
         raise RuntimeError("oracle_attention_rows failed: %d" % rc)
     return out, lse

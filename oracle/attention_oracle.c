@@ -64,6 +64,24 @@ double oracle_half_to_double(uint16_t h) { return half_bits_to_double(h); }
 /* rows: nrows triples (sequence, query head, row index inside the sequence).
  * Returns 0, or -1 if a routing group index would exceed 63, or -2 on a bad
  * row triple, or -3 if memory runs out. */
+/* An e4m3 code as a double: sign, 4 exponent bits (bias 7), 3 mantissa bits;
+ * exponent 0 is subnormal (m / 8 * 2^-6); exponent 15 with mantissa 7 is NaN. */
+static double e4m3_to_double(uint8_t c) {
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+    return sgn ? -v : v;
+}
+
+int oracle_attention_rows_fmt(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                              const int8_t* q8, const float* q_scale, const int8_t* k8,
+                              const float* k_scale, const uint64_t* masks, const int32_t* g,
+                              const int32_t* cu_seqlens, const int32_t* cu_qtiles,
+                              const int32_t* cu_ktiles, int nseq, int total_qtiles,
+                              int total_ktiles, int hq, int hk, int d, int causal,
+                              const int32_t* kv_map, double scale, const int64_t* rows,
+                              int64_t nrows, double* out, double* lse, int low_fp8);
+
 int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           const int8_t* q8, const float* q_scale, const int8_t* k8,
                           const float* k_scale, const uint64_t* masks, const int32_t* g,
@@ -72,6 +90,22 @@ int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* 
                           int total_ktiles, int hq, int hk, int d, int causal,
                           const int32_t* kv_map, double scale, const int64_t* rows,
                           int64_t nrows, double* out, double* lse) {
+    return oracle_attention_rows_fmt(q, k, v, q8, q_scale, k8, k_scale, masks, g, cu_seqlens,
+                                     cu_qtiles, cu_ktiles, nseq, total_qtiles, total_ktiles, hq,
+                                     hk, d, causal, kv_map, scale, rows, nrows, out, lse, 0);
+}
+
+/* As oracle_attention_rows; low_fp8 != 0 reads the codes as e4m3 values:
+ * a low-precision tile scores (sum_c e4m3(q8) * e4m3(k8)) * s_q * s_k * scale,
+ * exact in fp64 (products of two 4-significant-bit values, 128 of them). */
+int oracle_attention_rows_fmt(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                              const int8_t* q8, const float* q_scale, const int8_t* k8,
+                              const float* k_scale, const uint64_t* masks, const int32_t* g,
+                              const int32_t* cu_seqlens, const int32_t* cu_qtiles,
+                              const int32_t* cu_ktiles, int nseq, int total_qtiles,
+                              int total_ktiles, int hq, int hk, int d, int causal,
+                              const int32_t* kv_map, double scale, const int64_t* rows,
+                              int64_t nrows, double* out, double* lse, int low_fp8) {
     init_half_table();
     int max_len = 0;
     for (int s = 0; s < nseq; ++s) {
@@ -123,10 +157,17 @@ int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* 
                 double score;
                 if ((w >> b) & 1ULL) {
                     const int8_t* k8j = k8 + ((int64_t)(t0 + j) * hk + kv) * d;
-                    int64_t acc = 0;
-                    for (int c = 0; c < d; ++c) acc += (int64_t)q8i[c] * (int64_t)k8j[c];
                     double sk = (double)k_scale[(int64_t)kv * total_ktiles + cu_ktiles[s] + kt];
-                    score = (double)acc * sq * sk * scale;
+                    if (low_fp8) {
+                        double acc = 0.0;
+                        for (int c = 0; c < d; ++c)
+                            acc += e4m3_to_double((uint8_t)q8i[c]) * e4m3_to_double((uint8_t)k8j[c]);
+                        score = acc * sq * sk * scale;
+                    } else {
+                        int64_t acc = 0;
+                        for (int c = 0; c < d; ++c) acc += (int64_t)q8i[c] * (int64_t)k8j[c];
+                        score = (double)acc * sq * sk * scale;
+                    }
                 } else {
                     const uint16_t* kj = k + ((int64_t)(t0 + j) * hk + kv) * d;
                     double acc = 0.0;

@@ -731,3 +731,90 @@ def test_mass_probe_matches_python_loops():
                 assert abs(r["h8"][h, start + i] - h8) < 1e-10
         start += L
         cq += oracle.n_qtiles(L)
+
+
+# ------------------------------------------------------------- FP8 low path --
+from oracle import fp8 as of8  # noqa: E402
+
+
+def test_e4m3_table_fixed_points():
+    D = of8.DECODE
+    assert D[0x00] == 0.0 and D[0x80] == 0.0 and math.copysign(1, D[0x80]) < 0
+    assert D[0x01] == 2.0 ** -9                    # smallest subnormal
+    assert D[0x07] == 7 * 2.0 ** -9                # largest subnormal
+    assert D[0x08] == 2.0 ** -6                    # smallest normal
+    assert D[0x38] == 1.0 and D[0x40] == 2.0 and D[0x30] == 0.5
+    assert D[0x7E] == 448.0 and D[0xFE] == -448.0  # largest finite
+    assert math.isnan(D[0x7F]) and math.isnan(D[0xFF])
+    pos = D[:0x7F]
+    assert np.all(np.diff(pos) > 0)                # strictly increasing codes 0..0x7E
+    assert np.array_equal(D[0x80:0xFF], -pos)      # sign symmetry
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    pos = of8.DECODE[:0x7F]
+    codes = np.arange(0x7F, dtype=np.uint8)
+    assert np.array_equal(of8.e4m3_encode(pos.astype(np.float32)), codes)
+    assert np.array_equal(of8.e4m3_encode(-pos[1:].astype(np.float32)), codes[1:] | 0x80)
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)   # exact in fp32
+    assert np.all(mids.astype(np.float64) == (pos[:-1] + pos[1:]) / 2)
+    got = of8.e4m3_encode(mids).astype(int)
+    lower = np.arange(0x7E)
+    assert np.array_equal(got, np.where(lower % 2 == 0, lower, lower + 1))   # ties to even
+    just_above = np.nextafter(mids, np.float32(1000))
+    assert np.array_equal(of8.e4m3_encode(just_above).astype(int), lower + 1)
+    sat = of8.e4m3_encode(np.array([448.0, 463.9, 464.0, 1e6, -1e6], np.float32))
+    assert list(sat) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+
+
+def test_fp8_block_quantiser():
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((200, 2, 64)) * 3).astype(np.float16)
+    x[5, 1, 7] = np.float16(-40.0)                 # the block's absmax, negative
+    codes, sc = of8.quantize_blocks_fp8(x, [200], 64)
+    assert codes.dtype == np.uint8 and sc.shape == (2, 4)
+    assert sc[1, 0] == np.float32(40.0) / np.float32(448.0)
+    assert codes[5, 1, 7] == 0xFE                  # -absmax -> -448
+    back = of8.DECODE[codes] * sc[np.arange(2)[None, :, None], (np.arange(200) // 64)[:, None, None]]
+    err = np.abs(back - x.astype(np.float64))
+    # e4m3 keeps 3 mantissa bits: half an ulp is at most 2^-4 of the value
+    # (normal range); below 2^-6 s the subnormal spacing 2^-9 s bounds it
+    bound = np.maximum(np.abs(x.astype(np.float64)) * 2.0 ** -4,
+                       2.0 ** -10 * sc[np.arange(2)[None, :, None], (np.arange(200) // 64)[:, None, None]])
+    assert np.all(err <= bound * (1 + 1e-6))
+    z = np.zeros((10, 1, 64), np.float16)
+    c0, s0 = of8.quantize_blocks_fp8(z, [10], 64)
+    assert np.all(c0 == 0) and s0[0, 0] == 0.0
+
+
+def test_fp8_scale_exact_inputs_make_paths_agree():
+    # every block holds values whose ratio to the block scale is an exact e4m3
+    # value: the FP8 scores equal the FP16 scores, so all-FP8 routing gives
+    # the all-FP16 output
+    rng = np.random.default_rng(9)
+    lengths, hq, hk, d = [130, 64], 2, 1, 64
+    T = sum(lengths)
+    grid = of8.DECODE[rng.integers(0x30, 0x50, size=(T, hq + 2 * hk, d))]   # 0.5 .. 8, exact
+    sign = rng.choice([-1.0, 1.0], size=grid.shape)
+    vals = (grid * sign * 0.125).astype(np.float16)                        # exact in fp16
+    q, k = vals[:, :hq], vals[:, hq:hq + hk]
+    for blk_rows, arr in ((128, q), (64, k)):
+        start = 0
+        for L in lengths:
+            for b in range(0, L, blk_rows):
+                arr[start + b, :, 0] = np.float16(56.0)   # absmax 56 = 448 * 0.125 per block
+            start += L
+    v = rng.standard_normal((T, hk, d)).astype(np.float16)
+    q8, qs = of8.quantize_q_fp8(q, lengths)
+    k8, ks = of8.quantize_k_fp8(k, lengths)
+    assert np.all(qs[qs > 0] == np.float32(0.125)) and np.all(ks[ks > 0] == np.float32(0.125))
+    ones, _, _ = oracle.build_routing("band", 100, 0, lengths, hk, [1, 1], True)
+    zeros, _, _ = oracle.build_routing("band", 0, 0, lengths, hk, [1, 1], True)
+    o8, l8 = oracle.attention_rows(q, k, v, q8, qs, k8, ks, ones, [1, 1], lengths, True, low="fp8")
+    o16, l16 = oracle.attention_rows(q, k, v, q8, qs, k8, ks, zeros, [1, 1], lengths, True, low="fp8")
+    np.testing.assert_allclose(o8, o16, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l8, l16, rtol=0, atol=1e-12)
+    # and the INT8 reading of the same bytes differs (the flag is used)
+    oi, _ = oracle.attention_rows(q, k, v, q8.view(np.int8), qs, k8.view(np.int8), ks, ones,
+                                  [1, 1], lengths, True)
+    assert np.max(np.abs(oi - o16)) > 1e-3
