@@ -134,6 +134,20 @@ int tilemix_quantize_qk(const void* q_f16, const void* k_f16, const int32_t* cu_
                         int d, int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
                         void* stream);
 
+/* The FP8 low path's operands (an open alternative on the pages: "TileMix:
+ * Tile-Centric Mixed-Precision Attention for LLM Inference Acceleration",
+ * agihunt.info summary, limitations paragraph).  Same blocks, layouts and
+ * arguments as tilemix_quantize_qk; s = fp32(absmax / 448) and code =
+ * e4m3(fp32(x / s)) (IEEE division, round to nearest even, saturating to
+ * +-448), the e4m3 bytes stored in the int8 arrays; a zero block has s = 0
+ * and codes 0.  A tile routed to the low path then scores
+ * (sum_c e4m3(q) e4m3(k)) * s_q * s_k / sqrt(d) with fp32 accumulation. */
+int tilemix_quantize_qk_fp8(const void* q_f16, const void* k_f16, const int32_t* cu_seqlens_d,
+                            const int32_t* cu_qtiles_d, const int32_t* cu_ktiles_d, int nseq,
+                            int total_tokens, int total_qtiles, int total_ktiles, int hq, int hk,
+                            int d, int8_t* q_codes, float* q_scale, int8_t* k_codes,
+                            float* k_scale, void* stream);
+
 typedef struct tilemix_prefill_args {
   const void* q;          /* device fp16 [total_tokens][hq][d], 16-byte aligned */
   const void* k;          /* device fp16 [total_tokens][hk][d], 16-byte aligned */
@@ -166,6 +180,11 @@ typedef struct tilemix_prefill_args {
   void* event_kernel_begin;    /* NULL, or a cudaEvent_t recorded on `stream` just
                                   before the fused attention kernel ... */
   void* event_kernel_end;      /* ... and one recorded just after it (profiling) */
+  int low_format;              /* the low-precision path of bit-1 tiles: 0 = INT8
+                                  (the pages' method, default), 1 = FP8 e4m3 (see
+                                  tilemix_quantize_qk_fp8; k_i8 / k_scale, when given,
+                                  then hold e4m3 codes and their scales; no debug
+                                  INT32 dump) */
 } tilemix_prefill_args;
 
 /* Bytes of device workspace tilemix_prefill_fwd needs for these arguments

@@ -49,7 +49,11 @@ class PrefillArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("debug_int32_scores", ctypes.c_void_p),
         ("event_kernel_begin", ctypes.c_void_p), ("event_kernel_end", ctypes.c_void_p),
+        ("low_format", ctypes.c_int),
     ]
+
+
+LOW_FORMATS = {"int8": 0, "fp8": 1}
 
 
 class DecodeArgs(ctypes.Structure):
@@ -123,6 +127,8 @@ def lib():
         L.tilemix_build_routing.argtypes = [I, I, ctypes.c_uint64, P, I, I, P, I, P, P, P]
         L.tilemix_quantize_qk.restype = I
         L.tilemix_quantize_qk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P]
+        L.tilemix_quantize_qk_fp8.restype = I
+        L.tilemix_quantize_qk_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P]
         L.tilemix_workspace_size.restype = I
         L.tilemix_workspace_size.argtypes = [ctypes.POINTER(PrefillArgs),
                                              ctypes.POINTER(ctypes.c_size_t)]
@@ -230,10 +236,22 @@ def tilemix_quantize_qk(q, k, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_toke
            "tilemix_quantize_qk")
 
 
+def tilemix_quantize_qk_fp8(q, k, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_tokens,
+                            total_qtiles, total_ktiles, hq, hk, d, q_codes, q_scale, k_codes,
+                            k_scale, stream=None):
+    """The FP8 (e4m3) low path's codes (bytes in int8/uint8 tensors) and scales."""
+    _check(lib().tilemix_quantize_qk_fp8(_ptr(q), _ptr(k), _ptr(cu_seqlens), _ptr(cu_qtiles),
+                                         _ptr(cu_ktiles), int(nseq), int(total_tokens),
+                                         int(total_qtiles), int(total_ktiles), int(hq), int(hk),
+                                         int(d), _ptr(q_codes), _ptr(q_scale), _ptr(k_codes),
+                                         _ptr(k_scale), _stream_handle(stream)),
+           "tilemix_quantize_qk_fp8")
+
+
 def make_args(q, k, v, o, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_tokens, total_qtiles,
               total_ktiles, max_seqlen, masks, g, causal=True, softmax_scale=0.0,
               kv_head_of_q=None, lse=None, k_i8=None, k_scale=None, workspace=None,
-              debug_int32_scores=None, events=None) -> PrefillArgs:
+              debug_int32_scores=None, events=None, low="int8") -> PrefillArgs:
     T, hq, d = q.shape
     hk = k.shape[1]
     a = PrefillArgs()
@@ -261,6 +279,7 @@ def make_args(q, k, v, o, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_tokens, 
     if events is not None:  # (begin, end) torch.cuda.Event pair around the fused kernel
         a.event_kernel_begin = events[0].cuda_event
         a.event_kernel_end = events[1].cuda_event
+    a.low_format = LOW_FORMATS[low]
     return a
 
 
@@ -403,6 +422,7 @@ from .decode import TileMixDecode  # noqa: E402  (convenience wrapper)
 __all__ = [
     "BLOCK_M", "BLOCK_N", "DecodeArgs", "MAX_GROUPS", "PrefillArgs", "RouteArgs", "TEMPLATES",
     "TileMixError", "route_pooled", "tilemix_route_pooled", "tilemix_route_workspace_size",
+    "LOW_FORMATS", "tilemix_quantize_qk_fp8",
     "MassArgs", "mass_probe", "tilemix_mass_probe",
     "TileMixDecode", "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
     "tilemix_build_routing", "tilemix_decode_fwd", "tilemix_decode_workspace_size",

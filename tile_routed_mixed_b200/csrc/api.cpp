@@ -99,6 +99,8 @@ int check_args(const tilemix_prefill_args* a) {
   if (a->causal != 0 && a->causal != 1) return TILEMIX_ERR_INVALID_ARG;
   if (!(a->softmax_scale >= 0.f) || std::isinf(a->softmax_scale)) return TILEMIX_ERR_INVALID_ARG;
   if ((a->k_i8 == nullptr) != (a->k_scale == nullptr)) return TILEMIX_ERR_INVALID_ARG;
+  if (a->low_format != 0 && a->low_format != 1) return TILEMIX_ERR_INVALID_ARG;
+  if (a->low_format == 1 && a->debug_int32_scores) return TILEMIX_ERR_UNSUPPORTED;
   if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;  // nothing to do
   if (!a->q || !a->k || !a->v || !a->o || !a->cu_seqlens || !a->cu_qtiles || !a->cu_ktiles ||
       !a->masks || !a->g)
@@ -117,7 +119,7 @@ int quantize_impl(const void* q_f16, const void* k_f16,
                                     const int32_t* cu_ktiles_d, int nseq, int total_tokens,
                                     int total_qtiles, int total_ktiles, int hq, int hk, int d,
                                     int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
-                                    int* ticket, void* stream) {
+                                    int* ticket, int fp8, void* stream) {
   if (d != 64 && d != 128) return TILEMIX_ERR_UNSUPPORTED;
   if (nseq < 0 || total_tokens < 0 || total_qtiles < 0 || total_ktiles < 0)
     return TILEMIX_ERR_INVALID_ARG;
@@ -136,7 +138,7 @@ int quantize_impl(const void* q_f16, const void* k_f16,
   }
   if (tilemix::launch_quantize_qk(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq,
                                   total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8,
-                                  k_scale, ticket, st) != cudaSuccess)
+                                  k_scale, ticket, fp8, st) != cudaSuccess)
     return TILEMIX_ERR_CUDA;
   return TILEMIX_OK;
 }
@@ -169,7 +171,18 @@ TILEMIX_API int tilemix_quantize_qk(const void* q_f16, const void* k_f16,
                                     void* stream) {
   return quantize_impl(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq, total_tokens,
                        total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8, k_scale,
-                       nullptr, stream);
+                       nullptr, 0, stream);
+}
+
+TILEMIX_API int tilemix_quantize_qk_fp8(const void* q_f16, const void* k_f16,
+                                        const int32_t* cu_seqlens_d, const int32_t* cu_qtiles_d,
+                                        const int32_t* cu_ktiles_d, int nseq, int total_tokens,
+                                        int total_qtiles, int total_ktiles, int hq, int hk, int d,
+                                        int8_t* q_codes, float* q_scale, int8_t* k_codes,
+                                        float* k_scale, void* stream) {
+  return quantize_impl(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq, total_tokens,
+                       total_qtiles, total_ktiles, hq, hk, d, q_codes, q_scale, k_codes, k_scale,
+                       nullptr, 1, stream);
 }
 
 TILEMIX_API int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes) {
@@ -200,7 +213,7 @@ TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream)
   rc = quantize_impl(a->q, a->k_i8 ? nullptr : a->k, a->cu_seqlens, a->cu_qtiles, a->cu_ktiles,
                      a->nseq, a->total_tokens, a->total_qtiles, a->total_ktiles, a->hq, a->hk,
                      a->d, q8, q_scale, const_cast<int8_t*>(k8), const_cast<float*>(k_scale),
-                     ticket, stream);
+                     ticket, a->low_format, stream);
   if (rc != TILEMIX_OK) return rc;
 
   tilemix::PrefillParams p;
@@ -247,6 +260,7 @@ TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream)
   p.causal = a->causal;
   const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.low_fp8 = a->low_format;
   p.timeout_ns = wait_timeout_ns();
   if (a->event_kernel_begin &&
       cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_begin), st) != cudaSuccess)

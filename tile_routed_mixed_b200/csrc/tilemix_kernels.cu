@@ -10,6 +10,7 @@
 // Map: TileMix Routes INT8 Inside Dense Attention" (cognaptus.com, "The routing
 // mechanism is designed to stay inside the hot loop").
 #include <cuda.h>
+#include <cuda_fp8.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -79,9 +80,11 @@ struct QuantSide {
   int total_tiles, heads, block_rows;
 };
 
+// fp8 != 0: the FP8 low path's codes instead, e4m3(x / s) with s = a / 448
+// (round to nearest even, saturating; IEEE fp32 division for both).
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_qk_kernel(QuantSide qs, QuantSide ks, const int32_t* __restrict__ cu_seqlens,
-                       int nseq, int d, int* ticket) {
+                       int nseq, int d, int* ticket, int fp8) {
   if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;
   const int nq = qs.total_tiles * qs.heads;
   const bool is_q = static_cast<int>(blockIdx.x) < nq;
@@ -134,9 +137,30 @@ __global__ void __launch_bounds__(kQuantThreads)
   float a = red[0];
 #pragma unroll
   for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
-  const float s = __fdiv_rn(a, 127.0f);
+  const float s = __fdiv_rn(a, fp8 ? 448.0f : 127.0f);
   if (threadIdx.x == 0) scales[static_cast<size_t>(h) * total_tiles + tile] = s;
   const float r = a > 0.f ? __frcp_rn(s) : 0.f;
+  if (fp8) {
+#pragma unroll
+    for (int i = 0; i < kQuantChunks; ++i) {
+      const int c = threadIdx.x + i * kQuantThreads;
+      if (c < nchunks) {
+        uint32_t w[2] = {0u, 0u};
+        if (a > 0.f) {
+          const __half* hv = reinterpret_cast<const __half*>(&u[i]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t b8 = __nv_cvt_float_to_fp8(__fdiv_rn(__half2float(hv[e]), s),
+                                                      __NV_SATFINITE, __NV_E4M3);
+            w[e >> 2] |= b8 << (8 * (e & 3));
+          }
+        }
+        const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
+        *reinterpret_cast<uint2*>(codes + off) = make_uint2(w[0], w[1]);
+      }
+    }
+    return;
+  }
 
 #pragma unroll
   for (int i = 0; i < kQuantChunks; ++i) {
@@ -152,7 +176,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
                        int total_qtiles, int total_ktiles, int hq, int hk, int d, int8_t* q8,
-                       float* q_scale, int8_t* k8, float* k_scale, int* ticket,
+                       float* q_scale, int8_t* k8, float* k_scale, int* ticket, int fp8,
                        cudaStream_t stream) {
   QuantSide qs{static_cast<const __half*>(q), cu_qtiles, q8, q_scale, q ? total_qtiles : 0,
                hq, BM};
@@ -164,7 +188,7 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
     return ticket ? static_cast<int>(cudaMemsetAsync(ticket, 0, sizeof(int), stream)) : cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   quantize_qk_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-      qs, ks, cu_seqlens, nseq, d, ticket);
+      qs, ks, cu_seqlens, nseq, d, ticket, fp8);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -362,17 +386,25 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t tmpl, uint32_t addr) {
 
 // S = Q K^T of one 128 x 64 score tile into TMEM column d_s, in the precision
 // the routing bit selects.
-template <int D>
+// kFp8: the low-precision tiles are FP8 e4m3 (kind::f8f6f4, fp32 accumulate;
+// the descriptor's e4m3 formats are 0, like f16's) instead of INT8.
+template <int D, bool kFp8>
 __device__ __forceinline__ void issue_qk(uint32_t d_s, bool is_int, uint32_t aq16, uint32_t aq8,
                                          uint32_t bk16, uint32_t bk8, uint64_t tmpl16,
                                          uint64_t tmpl8) {
   constexpr uint32_t kIdF16 = ptx::idesc_f16(BM, BN, false);
   constexpr uint32_t kIdI8 = ptx::idesc_s8(BM, BN);
+  constexpr uint32_t kIdF8 = ptx::idesc_f16(BM, BN, false);
   if (is_int) {
 #pragma unroll
-    for (int k = 0; k < D / 32; ++k)
-      ptx::mma_i8_ss(d_s, desc_at(tmpl8, aq8 + k * 32), desc_at(tmpl8, bk8 + k * 32), kIdI8,
-                     k > 0 ? 1u : 0u);
+    for (int k = 0; k < D / 32; ++k) {
+      if constexpr (kFp8)
+        ptx::mma_f8_ss(d_s, desc_at(tmpl8, aq8 + k * 32), desc_at(tmpl8, bk8 + k * 32), kIdF8,
+                       k > 0 ? 1u : 0u);
+      else
+        ptx::mma_i8_ss(d_s, desc_at(tmpl8, aq8 + k * 32), desc_at(tmpl8, bk8 + k * 32), kIdI8,
+                       k > 0 ? 1u : 0u);
+    }
   } else {
 #pragma unroll
     for (int k = 0; k < D / 16; ++k)
@@ -481,7 +513,7 @@ struct RowState {
 // diagonal and sequence-tail tiles need, kDebug the INT32 score dump of debug
 // runs; the lean copy runs every other tile, so the hot loop carries no code
 // for them.  False if a wait gave up.
-template <int D, bool kMask, bool kDebug>
+template <int D, bool kMask, bool kDebug, bool kFp8>
 __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st, int i, bool is_int,
                                              uint32_t (&r)[64]) {
 #ifdef TILEMIX_TRACE
@@ -504,15 +536,16 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st,
   ++st.n_s;
   if (tr == 0) TRACE(11, q, i);
   const int key0 = i * BN;
-  if (kDebug && is_int && cx.p->dbg && cx.my_row < cx.L) {
+  if (kDebug && !kFp8 && is_int && cx.p->dbg && cx.my_row < cx.L) {
     int32_t* drow = cx.p->dbg +
                     (static_cast<size_t>(cx.h) * cx.p->total_tokens + cx.t0 + cx.my_row) * cx.p->dbg_cols;
     for (int j = 0; j < 64; ++j)
       if (key0 + j < cx.L) drow[key0 + j] = static_cast<int32_t>(r[j]);
   }
   // scores in the float domain, before the log2(e)-scaled softmax:
-  // FP16 tile: raw fp32 dot; INT8 tile: exact float of the INT32 dot.
-  if (is_int) {
+  // FP16 tile: raw fp32 dot; INT8 tile: exact float of the INT32 dot; FP8
+  // tile: the fp32 dot as it is.
+  if (!kFp8 && is_int) {
 #pragma unroll
     for (int j = 0; j < 64; ++j) r[j] = __float_as_uint(__int2float_rn(static_cast<int>(r[j])));
   }
@@ -596,7 +629,7 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st,
   return true;
 }
 
-template <int D>
+template <int D, bool kFp8>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ PrefillParams p) {
   using S = Smem<D>;
@@ -798,7 +831,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             if (i < ntq) {
               ptx::tc_fence_after();
               const int st = t % kStages;
-              issue_qk<D>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16 + st * S::kK16,
+              issue_qk<D, kFp8>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16 + st * S::kK16,
                           a_smem + S::kOffK8 + st * S::kK8, t16, t8);
               ptx::mma_commit(&bars->s_full[q]);
               ++n_s;
@@ -925,18 +958,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int i = 0;
       if (p.dbg) {
         for (; i < ntq; ++i, gc.next(gs))
-          if (!softmax_tile<D, true, true>(cx, st, i, gc.int8(word), r)) {
+          if (!softmax_tile<D, true, true, kFp8>(cx, st, i, gc.int8(word), r)) {
             ok = false;
             break;
           }
       }
       for (; ok && i < i_hot; ++i, gc.next(gs))
-        if (!softmax_tile<D, false, false>(cx, st, i, gc.int8(word), r)) {
+        if (!softmax_tile<D, false, false, kFp8>(cx, st, i, gc.int8(word), r)) {
           ok = false;
           break;
         }
       for (; ok && i < ntq; ++i, gc.next(gs))
-        if (!softmax_tile<D, true, false>(cx, st, i, gc.int8(word), r)) {
+        if (!softmax_tile<D, true, false, kFp8>(cx, st, i, gc.int8(word), r)) {
           ok = false;
           break;
         }
@@ -990,10 +1023,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (threadIdx.x == 0) CTA_TRACE(5, gtimer());
 }
 
-template <int D>
+template <int D, bool kFp8>
 static int launch_prefill_d(const PrefillParams& p, cudaStream_t stream) {
   const int smem = Smem<D>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D, kFp8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return static_cast<int>(e);
   const long long items = static_cast<long long>(p.max_qpairs) * p.nseq * p.hq;
@@ -1006,13 +1039,15 @@ static int launch_prefill_d(const PrefillParams& p, cudaStream_t stream) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return static_cast<int>(e);
   const unsigned blocks = static_cast<unsigned>(items < sms ? items : sms);
-  prefill_fwd_kernel<D><<<blocks, kPrefillThreads, smem, stream>>>(p);
+  prefill_fwd_kernel<D, kFp8><<<blocks, kPrefillThreads, smem, stream>>>(p);
   return static_cast<int>(cudaGetLastError());
 }
 
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_prefill_d<128>(p, stream);
-  if (d == 64) return launch_prefill_d<64>(p, stream);
+  if (d == 128) return p.low_fp8 ? launch_prefill_d<128, true>(p, stream)
+                                 : launch_prefill_d<128, false>(p, stream);
+  if (d == 64) return p.low_fp8 ? launch_prefill_d<64, true>(p, stream)
+                                : launch_prefill_d<64, false>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -12,7 +12,7 @@ from . import (BLOCK_M, make_args, tilemix_prefill_fwd, tilemix_tile_offsets,
 
 class TileMixPrefill:
     def __init__(self, lengths, hq, hk, d, masks, g, causal=True, softmax_scale=0.0,
-                 kv_head_of_q=None, device="cuda"):
+                 kv_head_of_q=None, device="cuda", low="int8"):
         self.lengths = [int(x) for x in lengths]
         self.hq, self.hk, self.d = int(hq), int(hk), int(d)
         cu = np.zeros(len(self.lengths) + 1, dtype=np.int32)
@@ -25,6 +25,7 @@ class TileMixPrefill:
         self.max_seqlen = max(self.lengths) if self.lengths else 0
         self.causal = bool(causal)
         self.softmax_scale = float(softmax_scale)
+        self.low = str(low)  # low-precision path of bit-1 tiles: "int8" or "fp8" (e4m3)
         self.device = torch.device(device)
         masks = np.ascontiguousarray(masks, dtype=np.uint64)
         if masks.shape != (self.total_qtiles, self.hk):
@@ -50,7 +51,7 @@ class TileMixPrefill:
                          self.max_seqlen, self.masks, self.g, causal=self.causal,
                          softmax_scale=self.softmax_scale, kv_head_of_q=self.kv_head_of_q,
                          lse=lse, k_i8=k_i8, k_scale=k_scale, workspace=self.workspace,
-                         debug_int32_scores=debug_int32_scores, events=events)
+                         debug_int32_scores=debug_int32_scores, events=events, low=self.low)
 
     def ensure_workspace(self, q, k, v, o, **kw):
         a = self.args(q, k, v, o, **kw)
