@@ -287,7 +287,7 @@ def bench_config(args, w, lengths, g):
             if len(set(lengths)) == 1 else "varlen", "hq": w["hq"], "hk": w["hk"],
             "head_dim": w["d"], "causal": w["causal"], "template": w["template"],
             "int8_percent": w["percent"], "g": g[0] if len(set(g)) == 1 else "per-sequence",
-            "block_m": 128, "block_n": 64,
+            "block_m": 128, "block_n": 64, "low_precision": getattr(args, "low", "int8"),
             "l2": "no flush: inputs and output (%.0f MB per step) exceed the 126 MB L2"
                   % (sum(lengths) * (2 * w["hq"] + 2 * w["hk"]) * w["d"] * 2 / 1e6)}
 
@@ -317,7 +317,7 @@ def run_gpu(args):
     cu = synth.cu_seqlens_of(lengths)
     masks, legal, int8 = tm.tilemix_build_routing(w["template"], w["percent"],
                                                   w["routing_seed"], cu, hk, g, causal)
-    pf = tm.TileMixPrefill(lengths, hq, hk, d, masks, g, causal=causal, device=dev)
+    pf = tm.TileMixPrefill(lengths, hq, hk, d, masks, g, causal=causal, device=dev, low=args.low)
     qd, kd, vd = (torch.from_numpy(x).to(dev) for x in (q, k, v))
     od = torch.empty_like(qd)
     pf.ensure_workspace(qd, kd, vd, od)
@@ -414,7 +414,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16+i8",
+        "dtype": "f16+i8" if args.low == "int8" else "f16+e4m3",
         "data": "synthetic",
         "config": bench_config(args, w, lengths, g),
         "roofline": {
@@ -935,6 +935,8 @@ def main():
     ap.add_argument("--workload", default="llama3b_4k_b8", choices=list(synth.WORKLOADS))
     ap.add_argument("--template", default=None)
     ap.add_argument("--percent", type=int, default=None)
+    ap.add_argument("--low", choices=["int8", "fp8"], default="int8",
+                    help="low-precision path of bit-1 tiles in the prefill bench (fp8 = e4m3)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=["prefill", "decode", "route", "mass"], default="prefill",
                     help="prefill (the headline metric), the decode step with the INT8 K "
