@@ -926,6 +926,46 @@ def run_mass(args):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------- mad path ---
+
+def run_mad(args):
+    """Mean absolute deviation of the GPU prefill output from the all-FP16
+    oracle (fp64) at each coverage of the workload's template, for INT8 and
+    FP8 low tiles, on sampled rows (every q-tile's first, middle and last row
+    of three heads plus random rows).  A report, not a timed bench line."""
+    import torch
+
+    import oracle
+    import tile_routed_mixed_b200 as tm
+    from oracle import fp8 as of8
+    from tests import gpu_cases as gc
+
+    w, lengths, g = workload(args.workload, args.template, args.percent)
+    case = gc.Case.workload(args.workload)
+    q, k, v = case.inputs()
+    rows = gc.sample_rows(case.lengths, case.hq, seed=3, per_head_random=16,
+                          heads={0, case.hq // 2, case.hq - 1}, tiles_per_head=16)
+    zero = case.masks(0)
+    q8, qs = oracle.quantize_q(q, case.lengths)
+    k8, ks = oracle.quantize_k(k, case.lengths)
+    ref, _ = oracle.attention_rows(q, k, v, q8, qs, k8, ks, zero, case.g, case.lengths,
+                                   case.causal, rows=rows)
+    qd, kd, vd = (torch.from_numpy(x).cuda() for x in (q, k, v))
+    out = {}
+    for low in ("int8", "fp8"):
+        for pct in (0, 10, 25, 50, 75, 100):
+            masks = oracle.build_routing(case.template, pct, case.routing_seed, case.lengths,
+                                         case.hk, case.g, case.causal)[0]
+            pf = tm.TileMixPrefill(case.lengths, case.hq, case.hk, case.d, masks, case.g,
+                                   causal=case.causal, low=low)
+            o = pf(qd, kd, vd).cpu().numpy()
+            got = gc.gather(case, o, rows).astype(np.float64)
+            out["%s_%d" % (low, pct)] = float(np.mean(np.abs(got - ref)))
+    print(json.dumps({"report": "mean abs deviation of the fp16 output from the all-FP16 oracle",
+                      "workload": args.workload, "template": case.template,
+                      "rows_sampled": int(rows.shape[0]), "mad": out}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -938,7 +978,8 @@ def main():
     ap.add_argument("--low", choices=["int8", "fp8"], default="int8",
                     help="low-precision path of bit-1 tiles in the prefill bench (fp8 = e4m3)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["prefill", "decode", "route", "mass"], default="prefill",
+    ap.add_argument("--path", choices=["prefill", "decode", "route", "mass", "mad"],
+                    default="prefill",
                     help="prefill (the headline metric), the decode step with the INT8 K "
                          "cache, or pooled-score adaptive routing")
     args = ap.parse_args()
@@ -950,6 +991,8 @@ def main():
         run_route(args)
     elif args.path == "mass":
         run_mass(args)
+    elif args.path == "mad":
+        run_mad(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
