@@ -228,6 +228,58 @@ int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
 #define TILEMIX_NOALLOC_SCRATCH_BYTES (64u << 20)
 int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
 
+/* Prefill from host memory, with the copies overlapped with the attention.
+ * (The TileMix pages have no counterpart: a deployment convenience of this
+ * library for inputs that arrive in host memory.)
+ *
+ * The batch is cut into at most `chunks` runs of whole sequences, each cut
+ * where the token count first reaches a further 1/chunks of the batch.  Per
+ * run: its q, k and v rows are copied host -> device on stream_in; once they
+ * landed, its quantisation and attention run on `stream` (the kernels of
+ * tilemix_prefill_fwd, restricted to the run's sequences); once those
+ * finished, its O rows are copied device -> host on stream_out.  So the
+ * upload of run c + 1 and the download of run c - 1 overlap the kernels of
+ * run c.  The uploads wait for everything enqueued on `stream` before the
+ * call, and `stream` waits for the last download, so work enqueued on
+ * `stream` after the call (an event, a synchronisation, the next call) sees
+ * o_h complete.  Results equal those of tilemix_prefill_fwd on the same
+ * inputs, bit for bit (every block's codes and every output row are computed
+ * the same way whichever run holds them).
+ *   dev           the device-side arguments, as for tilemix_prefill_fwd:
+ *                 dev.q, dev.k, dev.v, dev.o are device buffers of the whole
+ *                 batch (this call fills q, k, v and reads o back), the
+ *                 metadata arrays are on the device, dev.workspace is sized
+ *                 by tilemix_workspace_size(&dev); dev.lse, if given, stays on
+ *                 the device; dev.event_kernel_begin / end are not recorded
+ *   cu_seqlens_h  host [nseq + 1], the same offsets as dev.cu_seqlens
+ *   q_h           host fp16 [total_tokens][hq][d] (as dev.q) ...
+ *   k_h, v_h      host fp16 [total_tokens][hk][d] ...
+ *   o_h           host fp16 [total_tokens][hq][d] (output); the copies only
+ *                 overlap anything when these four are page-locked memory
+ *   chunks        >= 1, the most runs to cut the batch into (at most nseq)
+ *   stream_in, stream_out   two cudaStream_t, each different from `stream`
+ *   events        2 * chunks + 1 cudaEvent_t created by the caller (timing
+ *                 may be disabled), not in use by other work during the call
+ * INVALID_ARG also when a host pointer, a stream or `events` is NULL, chunks
+ * < 1, or cu_seqlens_h disagrees with total_tokens, total_qtiles,
+ * total_ktiles or max_seqlen (all checked before anything is enqueued);
+ * otherwise as tilemix_prefill_fwd.  On CUDA, part of the work may already
+ * be enqueued. */
+typedef struct tilemix_prefill_host_args {
+  tilemix_prefill_args dev;
+  const int32_t* cu_seqlens_h;
+  const void* q_h;
+  const void* k_h;
+  const void* v_h;
+  void* o_h;
+  int chunks;
+  void* stream_in;
+  void* stream_out;
+  void* events;               /* cudaEvent_t array [2 * chunks + 1] */
+} tilemix_prefill_host_args;
+
+int tilemix_prefill_host(const tilemix_prefill_host_args* args, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Decode with the INT8 K cache: one new query token per sequence.
  *

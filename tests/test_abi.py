@@ -145,6 +145,54 @@ def test_prefill_argument_checks_are_synchronous():
                                  None, None, None, None) == tm.ERR_UNSUPPORTED
 
 
+def test_prefill_host_argument_checks_are_synchronous():
+    """tilemix_prefill_host validates everything it reads on the host before
+    it enqueues anything (no device is touched by these calls)."""
+    L = tm.lib()
+    cu = np.array([0, 100, 256], dtype=np.int32)   # 2 sequences: 1 + 2 query tiles, 2 + 3 key tiles
+    events = (ctypes.c_void_p * 5)(*([4096] * 5))
+
+    def host(cu_arr=cu, **over):
+        h = tm.PrefillHostArgs()
+        h.dev = _fake_args(nseq=2, total_qtiles=3, total_ktiles=5, workspace=4096,
+                           workspace_bytes=1 << 30)
+        h.cu_seqlens_h = cu_arr.ctypes.data
+        h.q_h = h.k_h = h.v_h = h.o_h = 8192
+        h.chunks = 2
+        h.stream_in = h.stream_out = 16
+        h.events = ctypes.cast(events, ctypes.c_void_p).value
+        for k, v in over.items():
+            if k.startswith("dev_"):
+                setattr(h.dev, k[4:], v)
+            else:
+                setattr(h, k, v)
+        return h
+
+    assert L.tilemix_prefill_host(None, None) == tm.ERR_INVALID_ARG
+    cases = [
+        (dict(dev_d=96), tm.ERR_UNSUPPORTED),           # the device arguments' own checks
+        (dict(dev_q=None), tm.ERR_INVALID_ARG),
+        (dict(q_h=None), tm.ERR_INVALID_ARG),
+        (dict(o_h=None), tm.ERR_INVALID_ARG),
+        (dict(stream_in=None), tm.ERR_INVALID_ARG),
+        (dict(events=None), tm.ERR_INVALID_ARG),
+        (dict(chunks=0), tm.ERR_INVALID_ARG),
+        (dict(cu_seqlens_h=None), tm.ERR_INVALID_ARG),
+        (dict(dev_total_qtiles=4), tm.ERR_INVALID_ARG),  # disagrees with the host offsets
+        (dict(dev_total_ktiles=4), tm.ERR_INVALID_ARG),
+        (dict(dev_max_seqlen=155), tm.ERR_INVALID_ARG),  # shorter than sequence 1 (156)
+        (dict(dev_workspace=None), tm.ERR_WORKSPACE),
+    ]
+    for over, want in cases:
+        assert L.tilemix_prefill_host(ctypes.byref(host(**over)), None) == want, over
+    bad = np.array([0, 300, 256], dtype=np.int32)    # decreasing offsets
+    assert L.tilemix_prefill_host(ctypes.byref(host(bad)), None) == tm.ERR_INVALID_ARG
+    short = np.array([0, 100, 200], dtype=np.int32)  # ends before total_tokens
+    assert L.tilemix_prefill_host(ctypes.byref(host(short)), None) == tm.ERR_INVALID_ARG
+    # an empty batch is a no-op
+    assert L.tilemix_prefill_host(ctypes.byref(host(dev_nseq=0)), None) == tm.OK
+
+
 def _fake_decode(**over):
     a = tm.DecodeArgs()
     for f in ("q", "k", "v", "k_i8", "k_scale", "o", "seq_start", "seq_len", "ktile_start",

@@ -56,6 +56,17 @@ class PrefillArgs(ctypes.Structure):
 LOW_FORMATS = {"int8": 0, "fp8": 1}
 
 
+class PrefillHostArgs(ctypes.Structure):
+    """Mirror of ``tilemix_prefill_host_args``."""
+    _fields_ = [
+        ("dev", PrefillArgs), ("cu_seqlens_h", ctypes.c_void_p),
+        ("q_h", ctypes.c_void_p), ("k_h", ctypes.c_void_p), ("v_h", ctypes.c_void_p),
+        ("o_h", ctypes.c_void_p), ("chunks", ctypes.c_int),
+        ("stream_in", ctypes.c_void_p), ("stream_out", ctypes.c_void_p),
+        ("events", ctypes.c_void_p),
+    ]
+
+
 class DecodeArgs(ctypes.Structure):
     """Mirror of ``tilemix_decode_args``."""
     _fields_ = [
@@ -136,6 +147,8 @@ def lib():
         L.tilemix_prefill_fwd.argtypes = [ctypes.POINTER(PrefillArgs), P]
         L.tilemix_prefill_fwd_noalloc.restype = I
         L.tilemix_prefill_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), P]
+        L.tilemix_prefill_host.restype = I
+        L.tilemix_prefill_host.argtypes = [ctypes.POINTER(PrefillHostArgs), P]
         L.tilemix_decode_workspace_size.restype = I
         L.tilemix_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs),
                                                     ctypes.POINTER(ctypes.c_size_t)]
@@ -302,6 +315,12 @@ def tilemix_prefill_fwd_noalloc(args: PrefillArgs, stream=None):
            "tilemix_prefill_fwd_noalloc")
 
 
+def tilemix_prefill_host(args: PrefillHostArgs, stream=None):
+    """Host-buffer prefill with overlapped copies (see include/tilemix.h)."""
+    _check(lib().tilemix_prefill_host(ctypes.byref(args), _stream_handle(stream)),
+           "tilemix_prefill_host")
+
+
 def tilemix_selftest_wait_timeout(timeout_ms: int, stream=None):
     _check(lib().tilemix_selftest_wait_timeout(int(timeout_ms), _stream_handle(stream)),
            "tilemix_selftest_wait_timeout")
@@ -428,6 +447,7 @@ __all__ = [
     "tilemix_build_routing", "tilemix_decode_fwd", "tilemix_decode_workspace_size",
     "tilemix_get_error", "tilemix_prefill_fwd",
     "tilemix_prefill_fwd_noalloc", "tilemix_quantize_qk", "tilemix_selftest_wait_timeout",
+    "PrefillHostArgs", "tilemix_prefill_host",
     "tilemix_status_string", "tilemix_tile_offsets", "tilemix_version",
     "tilemix_workspace_size",
 ]

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -114,12 +115,11 @@ int check_args(const tilemix_prefill_args* a) {
 
 // Quantisation of the INT8 operands; a non-null ticket is zeroed by the
 // same launch.
-int quantize_impl(const void* q_f16, const void* k_f16,
-                                    const int32_t* cu_seqlens_d, const int32_t* cu_qtiles_d,
-                                    const int32_t* cu_ktiles_d, int nseq, int total_tokens,
-                                    int total_qtiles, int total_ktiles, int hq, int hk, int d,
-                                    int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
-                                    int* ticket, int fp8, void* stream) {
+int quantize_impl(const void* q_f16, const void* k_f16, const int32_t* cu_seqlens_d,
+                  const int32_t* cu_qtiles_d, const int32_t* cu_ktiles_d, int nseq,
+                  int total_tokens, const tilemix::QuantRange& range, int total_qtiles,
+                  int total_ktiles, int hq, int hk, int d, int8_t* q_i8, float* q_scale,
+                  int8_t* k_i8, float* k_scale, int* ticket, int fp8, void* stream) {
   if (d != 64 && d != 128) return TILEMIX_ERR_UNSUPPORTED;
   if (nseq < 0 || total_tokens < 0 || total_qtiles < 0 || total_ktiles < 0)
     return TILEMIX_ERR_INVALID_ARG;
@@ -137,8 +137,108 @@ int quantize_impl(const void* q_f16, const void* k_f16,
       return TILEMIX_ERR_INVALID_ARG;
   }
   if (tilemix::launch_quantize_qk(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq,
-                                  total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8,
-                                  k_scale, ticket, fp8, st) != cudaSuccess)
+                                  range, total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale,
+                                  k_i8, k_scale, ticket, fp8, st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  return TILEMIX_OK;
+}
+
+// What one prefill call shares between the runs of sequences it enqueues:
+// the workspace carve-up and the kernel parameters (tensor maps over the
+// whole batch's buffers).
+struct PrefillPlan {
+  tilemix::PrefillParams p;
+  int8_t* q8;
+  float* q_scale;
+  int8_t* k8;
+  float* k_scale;
+  int* ticket;
+  bool events;  // record event_kernel_begin / end around the attention launch
+};
+
+// Needs check_args(a) == OK and a non-empty batch.
+int plan_prefill(const tilemix_prefill_args* a, PrefillPlan* pl) {
+  const WorkspaceLayout w = layout_of(a);
+  if (!a->workspace || a->workspace_bytes < w.total ||
+      (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return TILEMIX_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  pl->q8 = reinterpret_cast<int8_t*>(ws + w.q8);
+  pl->q_scale = reinterpret_cast<float*>(ws + w.q_scale);
+  pl->k8 = a->k_i8 ? const_cast<int8_t*>(a->k_i8) : reinterpret_cast<int8_t*>(ws + w.k8);
+  pl->k_scale = a->k_i8 ? const_cast<float*>(a->k_scale) : reinterpret_cast<float*>(ws + w.k_scale);
+  pl->ticket = reinterpret_cast<int*>(ws + w.ticket);
+  pl->events = false;
+
+  tilemix::PrefillParams& p = pl->p;
+  std::memset(&p, 0, sizeof(p));
+  const int T = a->total_tokens, d = a->d;
+  int rc;
+  const CUtensorMapSwizzle sw8 =
+      d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if ((rc = encode_rows(&p.tm_q, a->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hq, d, 64,
+                        TILEMIX_BLOCK_M, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_q8, pl->q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a->hq, d, d,
+                        TILEMIX_BLOCK_M, sw8)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hk, d, 64,
+                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_k8, pl->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a->hk, d, d,
+                        TILEMIX_BLOCK_N, sw8)) != TILEMIX_OK)
+    return rc;
+  if ((rc = encode_rows(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hk, d, 64,
+                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
+    return rc;
+  p.o = a->o;
+  p.lse = a->lse;
+  p.kv_head_of_q = a->kv_head_of_q;
+  p.masks = a->masks;
+  p.q_scale = pl->q_scale;
+  p.k_scale = pl->k_scale;
+  p.dbg = a->debug_int32_scores;
+  p.ticket = pl->ticket;
+  p.dbg_cols = (a->max_seqlen + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N * TILEMIX_BLOCK_N;
+  p.total_tokens = T;
+  p.total_qtiles = a->total_qtiles;
+  p.total_ktiles = a->total_ktiles;
+  p.hq = a->hq;
+  p.hk = a->hk;
+  p.group = a->hq / a->hk;
+  p.causal = a->causal;
+  const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.low_fp8 = a->low_format;
+  p.timeout_ns = wait_timeout_ns();
+  return TILEMIX_OK;
+}
+
+// Quantisation and attention of sequences s0 .. s1 - 1 (their tiles `range`,
+// their longest sequence max_seqlen) on `st`.  Offsets stay absolute: the
+// sequence arrays are read from s0 on, every tensor and workspace array is
+// addressed as for the whole batch, so the runs of one call touch disjoint
+// rows and the same codes, scales and outputs come out as from one run.
+int run_prefill_range(const tilemix_prefill_args* a, PrefillPlan& pl, int s0, int s1,
+                      const tilemix::QuantRange& range, int max_seqlen, cudaStream_t st) {
+  int rc = quantize_impl(a->q, a->k_i8 ? nullptr : a->k, a->cu_seqlens + s0, a->cu_qtiles + s0,
+                         a->cu_ktiles + s0, s1 - s0, a->total_tokens, range, a->total_qtiles,
+                         a->total_ktiles, a->hq, a->hk, a->d, pl.q8, pl.q_scale, pl.k8,
+                         pl.k_scale, pl.ticket, a->low_format, st);
+  if (rc != TILEMIX_OK) return rc;
+  tilemix::PrefillParams p = pl.p;
+  p.cu_seqlens = a->cu_seqlens + s0;
+  p.cu_qtiles = a->cu_qtiles + s0;
+  p.cu_ktiles = a->cu_ktiles + s0;
+  p.g = a->g + s0;
+  p.nseq = s1 - s0;
+  p.max_qpairs = ((max_seqlen + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M + 1) / 2;
+  if (pl.events && a->event_kernel_begin &&
+      cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_begin), st) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  if (tilemix::launch_prefill(p, a->d, st) != cudaSuccess) return TILEMIX_ERR_CUDA;
+  if (pl.events && a->event_kernel_end &&
+      cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_end), st) != cudaSuccess)
     return TILEMIX_ERR_CUDA;
   return TILEMIX_OK;
 }
@@ -170,8 +270,8 @@ TILEMIX_API int tilemix_quantize_qk(const void* q_f16, const void* k_f16,
                                     int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
                                     void* stream) {
   return quantize_impl(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq, total_tokens,
-                       total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale, k_i8, k_scale,
-                       nullptr, 0, stream);
+                       {0, total_qtiles, 0, total_ktiles}, total_qtiles, total_ktiles, hq, hk, d,
+                       q_i8, q_scale, k_i8, k_scale, nullptr, 0, stream);
 }
 
 TILEMIX_API int tilemix_quantize_qk_fp8(const void* q_f16, const void* k_f16,
@@ -181,8 +281,8 @@ TILEMIX_API int tilemix_quantize_qk_fp8(const void* q_f16, const void* k_f16,
                                         int8_t* q_codes, float* q_scale, int8_t* k_codes,
                                         float* k_scale, void* stream) {
   return quantize_impl(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq, total_tokens,
-                       total_qtiles, total_ktiles, hq, hk, d, q_codes, q_scale, k_codes, k_scale,
-                       nullptr, 1, stream);
+                       {0, total_qtiles, 0, total_ktiles}, total_qtiles, total_ktiles, hq, hk, d,
+                       q_codes, q_scale, k_codes, k_scale, nullptr, 1, stream);
 }
 
 TILEMIX_API int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes) {
@@ -197,79 +297,12 @@ TILEMIX_API int tilemix_prefill_fwd(const tilemix_prefill_args* a, void* stream)
   int rc = check_args(a);
   if (rc != TILEMIX_OK) return rc;
   if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;
-  const WorkspaceLayout w = layout_of(a);
-  if (!a->workspace || a->workspace_bytes < w.total ||
-      (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
-    return TILEMIX_ERR_WORKSPACE;
+  PrefillPlan pl;
+  if ((rc = plan_prefill(a, &pl)) != TILEMIX_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
-  int8_t* q8 = reinterpret_cast<int8_t*>(ws + w.q8);
-  float* q_scale = reinterpret_cast<float*>(ws + w.q_scale);
-  const int8_t* k8 = a->k_i8 ? a->k_i8 : reinterpret_cast<int8_t*>(ws + w.k8);
-  const float* k_scale = a->k_i8 ? a->k_scale : reinterpret_cast<float*>(ws + w.k_scale);
-
-  // INT8 path operands: Q always, K unless the caller supplied its codes.
-  int* ticket = reinterpret_cast<int*>(ws + w.ticket);
-  rc = quantize_impl(a->q, a->k_i8 ? nullptr : a->k, a->cu_seqlens, a->cu_qtiles, a->cu_ktiles,
-                     a->nseq, a->total_tokens, a->total_qtiles, a->total_ktiles, a->hq, a->hk,
-                     a->d, q8, q_scale, const_cast<int8_t*>(k8), const_cast<float*>(k_scale),
-                     ticket, a->low_format, stream);
-  if (rc != TILEMIX_OK) return rc;
-
-  tilemix::PrefillParams p;
-  std::memset(&p, 0, sizeof(p));
-  const int T = a->total_tokens, d = a->d;
-  const CUtensorMapSwizzle sw8 =
-      d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if ((rc = encode_rows(&p.tm_q, a->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hq, d, 64,
-                        TILEMIX_BLOCK_M, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
-    return rc;
-  if ((rc = encode_rows(&p.tm_q8, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a->hq, d, d,
-                        TILEMIX_BLOCK_M, sw8)) != TILEMIX_OK)
-    return rc;
-  if ((rc = encode_rows(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hk, d, 64,
-                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
-    return rc;
-  if ((rc = encode_rows(&p.tm_k8, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a->hk, d, d,
-                        TILEMIX_BLOCK_N, sw8)) != TILEMIX_OK)
-    return rc;
-  if ((rc = encode_rows(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, a->hk, d, 64,
-                        TILEMIX_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B)) != TILEMIX_OK)
-    return rc;
-  p.o = a->o;
-  p.lse = a->lse;
-  p.cu_seqlens = a->cu_seqlens;
-  p.cu_qtiles = a->cu_qtiles;
-  p.cu_ktiles = a->cu_ktiles;
-  p.kv_head_of_q = a->kv_head_of_q;
-  p.masks = a->masks;
-  p.g = a->g;
-  p.q_scale = q_scale;
-  p.k_scale = k_scale;
-  p.dbg = a->debug_int32_scores;
-  p.ticket = ticket;
-  p.dbg_cols = (a->max_seqlen + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N * TILEMIX_BLOCK_N;
-  p.nseq = a->nseq;
-  p.total_tokens = T;
-  p.total_qtiles = a->total_qtiles;
-  p.total_ktiles = a->total_ktiles;
-  p.max_qpairs = ((a->max_seqlen + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M + 1) / 2;
-  p.hq = a->hq;
-  p.hk = a->hk;
-  p.group = a->hq / a->hk;
-  p.causal = a->causal;
-  const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.low_fp8 = a->low_format;
-  p.timeout_ns = wait_timeout_ns();
-  if (a->event_kernel_begin &&
-      cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_begin), st) != cudaSuccess)
-    return TILEMIX_ERR_CUDA;
-  if (tilemix::launch_prefill(p, d, st) != cudaSuccess) return TILEMIX_ERR_CUDA;
-  if (a->event_kernel_end &&
-      cudaEventRecord(static_cast<cudaEvent_t>(a->event_kernel_end), st) != cudaSuccess)
-    return TILEMIX_ERR_CUDA;
-  return TILEMIX_OK;
+  if (a->event_kernel_begin || a->event_kernel_end) pl.events = true;
+  return run_prefill_range(a, pl, 0, a->nseq, {0, a->total_qtiles, 0, a->total_ktiles},
+                           a->max_seqlen, st);
 }
 
 TILEMIX_API int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream) {
@@ -283,6 +316,88 @@ TILEMIX_API int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, vo
   a.workspace = scratch;
   a.workspace_bytes = TILEMIX_NOALLOC_SCRATCH_BYTES;
   return tilemix_prefill_fwd(&a, stream);
+}
+
+TILEMIX_API int tilemix_prefill_host(const tilemix_prefill_host_args* h, void* stream) {
+  if (!h) return TILEMIX_ERR_INVALID_ARG;
+  const tilemix_prefill_args* a = &h->dev;
+  int rc = check_args(a);
+  if (rc != TILEMIX_OK) return rc;
+  if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;
+  if (!h->cu_seqlens_h || !h->q_h || !h->k_h || !h->v_h || !h->o_h || !h->stream_in ||
+      !h->stream_out || !h->events || h->chunks < 1)
+    return TILEMIX_ERR_INVALID_ARG;
+  const int32_t* cu = h->cu_seqlens_h;
+  const int nseq = a->nseq;
+  if (cu[0] != 0 || cu[nseq] != a->total_tokens) return TILEMIX_ERR_INVALID_ARG;
+  // the device tile offsets must match the host token offsets
+  long long nq = 0, nk = 0;
+  for (int s = 0; s < nseq; ++s) {
+    const int L = cu[s + 1] - cu[s];
+    if (L < 0 || L > a->max_seqlen) return TILEMIX_ERR_INVALID_ARG;
+    nq += (L + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M;
+    nk += (L + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N;
+  }
+  if (nq != a->total_qtiles || nk != a->total_ktiles) return TILEMIX_ERR_INVALID_ARG;
+  const int chunks = h->chunks < nseq ? h->chunks : nseq;
+
+  PrefillPlan pl;
+  if ((rc = plan_prefill(a, &pl)) != TILEMIX_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t sin = static_cast<cudaStream_t>(h->stream_in);
+  cudaStream_t sout = static_cast<cudaStream_t>(h->stream_out);
+  cudaEvent_t* ev = static_cast<cudaEvent_t*>(h->events);
+  cudaEvent_t join = ev[2 * h->chunks];
+  const size_t qrow = static_cast<size_t>(a->hq) * a->d * 2;  // bytes per token
+  const size_t krow = static_cast<size_t>(a->hk) * a->d * 2;
+  auto at = [](const void* base, size_t off) {
+    return static_cast<void*>(static_cast<uint8_t*>(const_cast<void*>(base)) + off);
+  };
+  // uploads start once `stream` has finished what precedes this call (a
+  // previous call's kernels and downloads use the same device rows)
+  if (cudaEventRecord(join, st) != cudaSuccess || cudaStreamWaitEvent(sin, join, 0) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  // run c: whole sequences s0 .. s1 - 1, cut where the token count first
+  // reaches (c + 1) / chunks of the batch
+  int s0 = 0, q0 = 0, k0 = 0;
+  for (int c = 0; c < chunks && s0 < nseq; ++c) {
+    const long long target = static_cast<long long>(a->total_tokens) * (c + 1) / chunks;
+    int s1 = s0 + 1;
+    while (s1 < nseq && (c == chunks - 1 || cu[s1] < target)) ++s1;
+    int nqt = 0, nkt = 0, longest = 0;
+    for (int s = s0; s < s1; ++s) {
+      const int L = cu[s + 1] - cu[s];
+      nqt += (L + TILEMIX_BLOCK_M - 1) / TILEMIX_BLOCK_M;
+      nkt += (L + TILEMIX_BLOCK_N - 1) / TILEMIX_BLOCK_N;
+      longest = std::max(longest, L);
+    }
+    const size_t t0 = static_cast<size_t>(cu[s0]), n = static_cast<size_t>(cu[s1]) - t0;
+    if (n > 0) {
+      if (cudaMemcpyAsync(at(a->q, t0 * qrow), at(h->q_h, t0 * qrow), n * qrow,
+                          cudaMemcpyHostToDevice, sin) != cudaSuccess ||
+          cudaMemcpyAsync(at(a->k, t0 * krow), at(h->k_h, t0 * krow), n * krow,
+                          cudaMemcpyHostToDevice, sin) != cudaSuccess ||
+          cudaMemcpyAsync(at(a->v, t0 * krow), at(h->v_h, t0 * krow), n * krow,
+                          cudaMemcpyHostToDevice, sin) != cudaSuccess ||
+          cudaEventRecord(ev[2 * c], sin) != cudaSuccess ||
+          cudaStreamWaitEvent(st, ev[2 * c], 0) != cudaSuccess)
+        return TILEMIX_ERR_CUDA;
+      rc = run_prefill_range(a, pl, s0, s1, {q0, nqt, k0, nkt}, longest, st);
+      if (rc != TILEMIX_OK) return rc;
+      if (cudaEventRecord(ev[2 * c + 1], st) != cudaSuccess ||
+          cudaStreamWaitEvent(sout, ev[2 * c + 1], 0) != cudaSuccess ||
+          cudaMemcpyAsync(at(h->o_h, t0 * qrow), at(a->o, t0 * qrow), n * qrow,
+                          cudaMemcpyDeviceToHost, sout) != cudaSuccess)
+        return TILEMIX_ERR_CUDA;
+    }
+    s0 = s1;
+    q0 += nqt;
+    k0 += nkt;
+  }
+  // `stream` ends with the last download
+  if (cudaEventRecord(join, sout) != cudaSuccess || cudaStreamWaitEvent(st, join, 0) != cudaSuccess)
+    return TILEMIX_ERR_CUDA;
+  return TILEMIX_OK;
 }
 
 namespace {

@@ -111,11 +111,18 @@ int launch_decode(const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_beg
 // One launch quantises Q (128-row blocks) and K (64-row blocks); a null q or
 // k skips that side.  A non-null ticket is set to zero by the same launch
 // (the fused kernel that follows on the stream hands out work from it).
+// Tiles a quantisation launch covers: Q tiles qtile0 .. qtile0 + nqtiles - 1
+// and K tiles ktile0 .. ktile0 + nktiles - 1, those of the nseq sequences
+// whose offsets cu_seqlens / cu_qtiles / cu_ktiles point at (a whole batch, or
+// a run of its sequences with the pointers advanced to the run's first).
+struct QuantRange {
+  int qtile0, nqtiles, ktile0, nktiles;
+};
 int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
-                       int total_qtiles, int total_ktiles, int hq, int hk, int d, int8_t* q8,
-                       float* q_scale, int8_t* k8, float* k_scale, int* ticket, int fp8,
-                       cudaStream_t stream);
+                       const QuantRange& range, int total_qtiles, int total_ktiles, int hq,
+                       int hk, int d, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                       int* ticket, int fp8, cudaStream_t stream);
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
 int read_and_clear_status(unsigned int* status, cudaStream_t stream);
 // Device address of the allocation-free entry point's scratch array on the

@@ -72,12 +72,14 @@ constexpr int BN = 64;   // keys per tile
 constexpr int kQuantThreads = 256;
 constexpr int kQuantChunks = 8;  // per thread: 128 rows x 128 dims / 8 / 256
 
+// One tensor's blocks: tiles tile0 .. tile0 + ntiles - 1 (cu_tiles holds the
+// sequences' first tiles, cu_tiles[0] <= tile0), scales [heads][total_tiles].
 struct QuantSide {
   const __half* x;
   const int32_t* cu_tiles;
   int8_t* codes;
   float* scales;
-  int total_tiles, heads, block_rows;
+  int tile0, ntiles, total_tiles, heads, block_rows;
 };
 
 // fp8 != 0: the FP8 low path's codes instead, e4m3(x / s) with s = a / 448
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     quantize_qk_kernel(QuantSide qs, QuantSide ks, const int32_t* __restrict__ cu_seqlens,
                        int nseq, int d, int* ticket, int fp8) {
   if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;
-  const int nq = qs.total_tiles * qs.heads;
+  const int nq = qs.ntiles * qs.heads;
   const bool is_q = static_cast<int>(blockIdx.x) < nq;
   // field-wise selection keeps both parameter structs in the constant bank
   const __half* x = is_q ? qs.x : ks.x;
@@ -97,8 +99,9 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int heads = is_q ? qs.heads : ks.heads;
   const int block_rows = is_q ? qs.block_rows : ks.block_rows;
   const int b = is_q ? blockIdx.x : blockIdx.x - nq;
-  const int tile = b / heads;
-  const int h = b - tile * heads;
+  const int rel = b / heads;
+  const int h = b - rel * heads;
+  const int tile = (is_q ? qs.tile0 : ks.tile0) + rel;
   // owning sequence: last s with cu_tiles[s] <= tile
   int lo = 0, hi = nseq - 1;
   while (lo < hi) {
@@ -175,15 +178,15 @@ __global__ void __launch_bounds__(kQuantThreads)
 
 int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
-                       int total_qtiles, int total_ktiles, int hq, int hk, int d, int8_t* q8,
-                       float* q_scale, int8_t* k8, float* k_scale, int* ticket, int fp8,
-                       cudaStream_t stream) {
-  QuantSide qs{static_cast<const __half*>(q), cu_qtiles, q8, q_scale, q ? total_qtiles : 0,
-               hq, BM};
-  QuantSide ks{static_cast<const __half*>(k), cu_ktiles, k8, k_scale, k ? total_ktiles : 0,
-               hk, BN};
-  const long long blocks = static_cast<long long>(qs.total_tiles) * hq +
-                           static_cast<long long>(ks.total_tiles) * hk;
+                       const QuantRange& range, int total_qtiles, int total_ktiles, int hq,
+                       int hk, int d, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                       int* ticket, int fp8, cudaStream_t stream) {
+  QuantSide qs{static_cast<const __half*>(q), cu_qtiles, q8, q_scale, range.qtile0,
+               q ? range.nqtiles : 0, total_qtiles, hq, BM};
+  QuantSide ks{static_cast<const __half*>(k), cu_ktiles, k8, k_scale, range.ktile0,
+               k ? range.nktiles : 0, total_ktiles, hk, BN};
+  const long long blocks = static_cast<long long>(qs.ntiles) * hq +
+                           static_cast<long long>(ks.ntiles) * hk;
   if (blocks == 0)
     return ticket ? static_cast<int>(cudaMemsetAsync(ticket, 0, sizeof(int), stream)) : cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

@@ -6,8 +6,10 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (BLOCK_M, make_args, tilemix_prefill_fwd, tilemix_tile_offsets,
-               tilemix_workspace_size)
+import ctypes
+
+from . import (BLOCK_M, PrefillHostArgs, make_args, tilemix_prefill_fwd, tilemix_prefill_host,
+               tilemix_tile_offsets, tilemix_workspace_size)
 
 
 class TileMixPrefill:
@@ -39,6 +41,8 @@ class TileMixPrefill:
         self.kv_head_of_q = (None if kv_head_of_q is None else
                              torch.as_tensor(np.asarray(kv_head_of_q, dtype=np.int32)).to(self.device))
         self.workspace = None
+        self.cu_host = cu
+        self._host_side = None  # (chunks, stream_in, stream_out, events, handle array)
 
     @property
     def max_qtiles(self):
@@ -66,3 +70,37 @@ class TileMixPrefill:
         self.ensure_workspace(q, k, v, o, lse=lse, **kw)
         tilemix_prefill_fwd(self.args(q, k, v, o, lse=lse, **kw), stream)
         return o
+
+    def host_args(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8):
+        """Arguments of ``tilemix_prefill_host``: host tensors q_h, k_h, v_h, o_h
+        (page-locked for the copies to overlap) and the device buffers q, k, v,
+        o of the same shapes.  The side streams and events are kept here."""
+        for name, t in (("q_h", q_h), ("k_h", k_h), ("v_h", v_h), ("o_h", o_h)):
+            if t.device.type != "cpu" or not t.is_contiguous() or t.dtype != torch.float16:
+                raise ValueError("%s must be a contiguous fp16 CPU tensor" % name)
+        chunks = int(chunks)
+        if self._host_side is None or self._host_side[0] != chunks:
+            s_in = torch.cuda.Stream(device=self.device)
+            s_out = torch.cuda.Stream(device=self.device)
+            evs = [torch.cuda.Event() for _ in range(2 * chunks + 1)]
+            for e in evs:  # creates the CUDA event
+                e.record(s_in)
+            handles = (ctypes.c_void_p * len(evs))(*[e.cuda_event for e in evs])
+            self._host_side = (chunks, s_in, s_out, evs, handles)
+        _, s_in, s_out, _, handles = self._host_side
+        self.ensure_workspace(q, k, v, o)
+        h = PrefillHostArgs()
+        h.dev = self.args(q, k, v, o)
+        h.cu_seqlens_h = self.cu_host.ctypes.data
+        h.q_h, h.k_h, h.v_h, h.o_h = (t.data_ptr() for t in (q_h, k_h, v_h, o_h))
+        h.chunks = chunks
+        h.stream_in = s_in.cuda_stream
+        h.stream_out = s_out.cuda_stream
+        h.events = ctypes.cast(handles, ctypes.c_void_p).value
+        return h
+
+    def from_host(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8, stream=None):
+        """O of host inputs into host o_h through tilemix_prefill_host; work
+        enqueued on `stream` afterwards sees o_h complete."""
+        tilemix_prefill_host(self.host_args(q_h, k_h, v_h, o_h, q, k, v, o, chunks), stream)
+        return o_h
