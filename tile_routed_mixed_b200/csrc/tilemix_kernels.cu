@@ -1,16 +1,17 @@
 // CUDA kernels of the tile-routed FP16/INT8 causal prefill attention (sm_100a).
 //
-//   quantize_qk_kernel       per-(head, block) symmetric absmax/127 INT8 codes
 //   prefill_fwd_kernel       fused attention: TMA -> tcgen05 kind::f16 or
 //                            kind::i8 QK^T per key tile (chosen by the routing
 //                            bit) -> shared online softmax -> kind::f16 P.V
+//   decode_attn_kernel       one new query row per sequence against the INT8 K
+//                            cache (tilemix_decode.cuh, included at the end)
+// The block quantiser that feeds both is in tilemix_quantize.cu.
 //
 // Method: "TileMix: Tile-Centric Mixed-Precision Attention for LLM Inference
 // Acceleration" (agihunt.info summary, method paragraphs) and "Precision Has a
 // Map: TileMix Routes INT8 Inside Dense Attention" (cognaptus.com, "The routing
 // mechanism is designed to stay inside the hot loop").
 #include <cuda.h>
-#include <cuda_fp8.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -60,140 +61,6 @@ __device__ __forceinline__ unsigned long long gtimer() {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 64;   // keys per tile
-
-// ===================================================================
-// Block quantisation ("only Q and K are quantised, Q in 128 x d blocks and K
-// in 64 x d blocks, symmetric absmax / 127").  One launch covers every Q block
-// and every K block; one CTA per (block, head) holds its block in registers
-// (at most eight 16-byte chunks per thread), so HBM sees each fp16 element
-// read once and each code written once.  codes = clamp(rne(x / s), +-127)
-// with s = a / 127, both divisions IEEE fp32.
-// ===================================================================
-constexpr int kQuantThreads = 256;
-constexpr int kQuantChunks = 8;  // per thread: 128 rows x 128 dims / 8 / 256
-
-// One tensor's blocks: tiles tile0 .. tile0 + ntiles - 1 (cu_tiles holds the
-// sequences' first tiles, cu_tiles[0] <= tile0), scales [heads][total_tiles].
-struct QuantSide {
-  const __half* x;
-  const int32_t* cu_tiles;
-  int8_t* codes;
-  float* scales;
-  int tile0, ntiles, total_tiles, heads, block_rows;
-};
-
-// fp8 != 0: the FP8 low path's codes instead, e4m3(x / s) with s = a / 448
-// (round to nearest even, saturating; IEEE fp32 division for both).
-__global__ void __launch_bounds__(kQuantThreads)
-    quantize_qk_kernel(QuantSide qs, QuantSide ks, const int32_t* __restrict__ cu_seqlens,
-                       int nseq, int d, int* ticket, int fp8) {
-  if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;
-  const int nq = qs.ntiles * qs.heads;
-  const bool is_q = static_cast<int>(blockIdx.x) < nq;
-  // field-wise selection keeps both parameter structs in the constant bank
-  const __half* x = is_q ? qs.x : ks.x;
-  const int32_t* cu_tiles = is_q ? qs.cu_tiles : ks.cu_tiles;
-  int8_t* codes = is_q ? qs.codes : ks.codes;
-  float* scales = is_q ? qs.scales : ks.scales;
-  const int total_tiles = is_q ? qs.total_tiles : ks.total_tiles;
-  const int heads = is_q ? qs.heads : ks.heads;
-  const int block_rows = is_q ? qs.block_rows : ks.block_rows;
-  const int b = is_q ? blockIdx.x : blockIdx.x - nq;
-  const int rel = b / heads;
-  const int h = b - rel * heads;
-  const int tile = (is_q ? qs.tile0 : ks.tile0) + rel;
-  // owning sequence: last s with cu_tiles[s] <= tile
-  int lo = 0, hi = nseq - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(cu_tiles + mid) <= tile) lo = mid; else hi = mid - 1;
-  }
-  const int t0 = __ldg(cu_seqlens + lo);
-  const int L = __ldg(cu_seqlens + lo + 1) - t0;
-  const int r0 = (tile - __ldg(cu_tiles + lo)) * block_rows;
-  const int rows = min(block_rows, L - r0);
-  const int cpr_log2 = d == 128 ? 4 : 3;  // 16-byte chunks per row
-  const int nchunks = rows << cpr_log2;
-  const size_t row_stride = static_cast<size_t>(heads) * d;
-  const size_t base = (static_cast<size_t>(t0 + r0) * heads + h) * d;
-
-  uint4 u[kQuantChunks];
-  __half2 amax2 = __float2half2_rn(0.f);
-#pragma unroll
-  for (int i = 0; i < kQuantChunks; ++i) {
-    const int c = threadIdx.x + i * kQuantThreads;
-    u[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (c < nchunks) {
-      const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
-      u[i] = *reinterpret_cast<const uint4*>(x + off);
-    }
-    const __half2* hv = reinterpret_cast<const __half2*>(&u[i]);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) amax2 = __hmax2(amax2, __habs2(hv[k]));
-  }
-  float amax = fmaxf(__low2float(amax2), __high2float(amax2));
-  __shared__ float red[kQuantThreads / 32];
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-  __syncthreads();
-  float a = red[0];
-#pragma unroll
-  for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
-  const float s = __fdiv_rn(a, fp8 ? 448.0f : 127.0f);
-  if (threadIdx.x == 0) scales[static_cast<size_t>(h) * total_tiles + tile] = s;
-  const float r = a > 0.f ? __frcp_rn(s) : 0.f;
-  if (fp8) {
-#pragma unroll
-    for (int i = 0; i < kQuantChunks; ++i) {
-      const int c = threadIdx.x + i * kQuantThreads;
-      if (c < nchunks) {
-        uint32_t w[2] = {0u, 0u};
-        if (a > 0.f) {
-          const __half* hv = reinterpret_cast<const __half*>(&u[i]);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t b8 = __nv_cvt_float_to_fp8(__fdiv_rn(__half2float(hv[e]), s),
-                                                      __NV_SATFINITE, __NV_E4M3);
-            w[e >> 2] |= b8 << (8 * (e & 3));
-          }
-        }
-        const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
-        *reinterpret_cast<uint2*>(codes + off) = make_uint2(w[0], w[1]);
-      }
-    }
-    return;
-  }
-
-#pragma unroll
-  for (int i = 0; i < kQuantChunks; ++i) {
-    const int c = threadIdx.x + i * kQuantThreads;
-    if (c < nchunks) {
-      const uint2 packed = a > 0.f ? quant_chunk(u[i], s, r) : make_uint2(0u, 0u);
-      const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
-      *reinterpret_cast<uint2*>(codes + off) = packed;
-    }
-  }
-}
-
-int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
-                       const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
-                       const QuantRange& range, int total_qtiles, int total_ktiles, int hq,
-                       int hk, int d, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
-                       int* ticket, int fp8, cudaStream_t stream) {
-  QuantSide qs{static_cast<const __half*>(q), cu_qtiles, q8, q_scale, range.qtile0,
-               q ? range.nqtiles : 0, total_qtiles, hq, BM};
-  QuantSide ks{static_cast<const __half*>(k), cu_ktiles, k8, k_scale, range.ktile0,
-               k ? range.nktiles : 0, total_ktiles, hk, BN};
-  const long long blocks = static_cast<long long>(qs.ntiles) * hq +
-                           static_cast<long long>(ks.ntiles) * hk;
-  if (blocks == 0)
-    return ticket ? static_cast<int>(cudaMemsetAsync(ticket, 0, sizeof(int), stream)) : cudaSuccess;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  quantize_qk_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-      qs, ks, cu_seqlens, nseq, d, ticket, fp8);
-  return static_cast<int>(cudaGetLastError());
-}
 
 // ===================================================================
 // Fused attention forward.
