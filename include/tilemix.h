@@ -239,12 +239,13 @@ int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
  * tilemix_prefill_fwd, restricted to the run's sequences); once those
  * finished, its O rows are copied device -> host on stream_out.  So the
  * upload of run c + 1 and the download of run c - 1 overlap the kernels of
- * run c.  The uploads wait for everything enqueued on `stream` before the
- * call, and `stream` waits for the last download, so work enqueued on
- * `stream` after the call (an event, a synchronisation, the next call) sees
- * o_h complete.  Results equal those of tilemix_prefill_fwd on the same
- * inputs, bit for bit (every block's codes and every output row are computed
- * the same way whichever run holds them).
+ * run c.  Unless after_previous is set, the uploads wait for everything
+ * enqueued on `stream` before the call.  `stream` waits for the last
+ * download, so work enqueued on `stream` after the call (an event, a
+ * synchronisation, the next call) sees o_h complete.  Results equal those
+ * of tilemix_prefill_fwd on the same inputs, bit for bit (every block's
+ * codes and every output row are computed the same way whichever run holds
+ * them).
  *   dev           the device-side arguments, as for tilemix_prefill_fwd:
  *                 dev.q, dev.k, dev.v, dev.o are device buffers of the whole
  *                 batch (this call fills q, k, v and reads o back), the
@@ -258,10 +259,21 @@ int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
  *                 overlap anything when these four are page-locked memory
  *   chunks        >= 1, the most runs to cut the batch into (at most nseq)
  *   stream_in, stream_out   two cudaStream_t, each different from `stream`
- *   events        2 * chunks + 1 cudaEvent_t created by the caller (timing
- *                 may be disabled), not in use by other work during the call
+ *   events        3 * chunks + 1 cudaEvent_t created by the caller (timing
+ *                 may be disabled), used by nothing else: per run, its
+ *                 upload, kernels and download are recorded in events
+ *                 3c, 3c + 1 and 3c + 2 (the last event joins the streams)
+ *   after_previous  0, or 1 when this call follows one made with the same
+ *                 events array, device buffers, batch and chunks (a stream
+ *                 of batches): run c's upload then waits only for that
+ *                 call's kernels of run c, and run c's kernels for its
+ *                 download of run c, so this batch's uploads start while
+ *                 the previous batch finishes; nothing else enqueued on
+ *                 `stream` before the call is waited for by the uploads.
+ *                 (Run c's waits on events 3c + 1 and 3c + 2 are made in
+ *                 both modes; an event never recorded is no wait.)
  * INVALID_ARG also when a host pointer, a stream or `events` is NULL, chunks
- * < 1, or cu_seqlens_h disagrees with total_tokens, total_qtiles,
+ * < 1, after_previous not 0 or 1, or cu_seqlens_h disagrees with total_tokens, total_qtiles,
  * total_ktiles or max_seqlen (all checked before anything is enqueued);
  * otherwise as tilemix_prefill_fwd.  On CUDA, part of the work may already
  * be enqueued. */
@@ -275,7 +287,8 @@ typedef struct tilemix_prefill_host_args {
   int chunks;
   void* stream_in;
   void* stream_out;
-  void* events;               /* cudaEvent_t array [2 * chunks + 1] */
+  void* events;               /* cudaEvent_t array [3 * chunks + 1] */
+  int after_previous;
 } tilemix_prefill_host_args;
 
 int tilemix_prefill_host(const tilemix_prefill_host_args* args, void* stream);

@@ -150,7 +150,7 @@ def test_prefill_host_argument_checks_are_synchronous():
     it enqueues anything (no device is touched by these calls)."""
     L = tm.lib()
     cu = np.array([0, 100, 256], dtype=np.int32)   # 2 sequences: 1 + 2 query tiles, 2 + 3 key tiles
-    events = (ctypes.c_void_p * 5)(*([4096] * 5))
+    events = (ctypes.c_void_p * 7)(*([4096] * 7))
 
     def host(cu_arr=cu, **over):
         h = tm.PrefillHostArgs()
@@ -177,6 +177,7 @@ def test_prefill_host_argument_checks_are_synchronous():
         (dict(stream_in=None), tm.ERR_INVALID_ARG),
         (dict(events=None), tm.ERR_INVALID_ARG),
         (dict(chunks=0), tm.ERR_INVALID_ARG),
+        (dict(after_previous=2), tm.ERR_INVALID_ARG),
         (dict(cu_seqlens_h=None), tm.ERR_INVALID_ARG),
         (dict(dev_total_qtiles=4), tm.ERR_INVALID_ARG),  # disagrees with the host offsets
         (dict(dev_total_ktiles=4), tm.ERR_INVALID_ARG),

@@ -71,6 +71,40 @@ def test_host_prefill_back_to_back_calls():
     assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
 
 
+def test_host_prefill_chained_calls_keep_each_batch():
+    """Calls chained with after_previous reuse the device rows while the
+    previous batch is still in flight: each batch's uploads wait only for the
+    previous batch's kernels of the same run.  Three different batches, each
+    downloaded into its own host buffer, must each equal its own device
+    result."""
+    import tile_routed_mixed_b200 as tm
+    case = CASES[0][1]
+    masks = case.masks()
+    batches = []
+    for seed in (11, 12, 13):
+        c = gc.Case(case.lengths, case.hq, case.hk, case.d, template=case.template,
+                    percent=case.percent, outliers=case.outliers, seed=seed)
+        q, k, v = c.inputs()
+        batches.append((q, k, v, gc.run_gpu(c, q, k, v, masks)["o"]))
+    pf = tm.TileMixPrefill(case.lengths, case.hq, case.hk, case.d, masks, case.g,
+                           causal=case.causal)
+    shape_q, shape_k = batches[0][0].shape, batches[0][1].shape
+    qd = torch.empty(shape_q, dtype=torch.float16, device="cuda")
+    kd = torch.empty(shape_k, dtype=torch.float16, device="cuda")
+    vd = torch.empty(shape_k, dtype=torch.float16, device="cuda")
+    od = torch.empty(shape_q, dtype=torch.float16, device="cuda")
+    hosts = []
+    for i, (q, k, v, _) in enumerate(batches):
+        qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+        oh = torch.full(shape_q, float("nan"), dtype=torch.float16).pin_memory()
+        hosts.append((qh, kh, vh, oh))
+        pf.from_host(qh, kh, vh, oh, qd, kd, vd, od, chunks=3, after_previous=i > 0)
+    torch.cuda.current_stream().synchronize()
+    assert tm.tilemix_get_error() == tm.OK
+    for (_, _, _, want), (_, _, _, oh) in zip(batches, hosts):
+        assert np.array_equal(oh.numpy().view(np.uint16), want.view(np.uint16))
+
+
 def test_host_prefill_workload_equals_device_call():
     """The 4k x b8 benchmark workload (one sequence per run), bit for bit
     against the device-buffer call."""

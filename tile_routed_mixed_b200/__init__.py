@@ -63,7 +63,7 @@ class PrefillHostArgs(ctypes.Structure):
         ("q_h", ctypes.c_void_p), ("k_h", ctypes.c_void_p), ("v_h", ctypes.c_void_p),
         ("o_h", ctypes.c_void_p), ("chunks", ctypes.c_int),
         ("stream_in", ctypes.c_void_p), ("stream_out", ctypes.c_void_p),
-        ("events", ctypes.c_void_p),
+        ("events", ctypes.c_void_p), ("after_previous", ctypes.c_int),
     ]
 
 

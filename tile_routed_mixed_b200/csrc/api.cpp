@@ -325,7 +325,8 @@ TILEMIX_API int tilemix_prefill_host(const tilemix_prefill_host_args* h, void* s
   if (rc != TILEMIX_OK) return rc;
   if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;
   if (!h->cu_seqlens_h || !h->q_h || !h->k_h || !h->v_h || !h->o_h || !h->stream_in ||
-      !h->stream_out || !h->events || h->chunks < 1)
+      !h->stream_out || !h->events || h->chunks < 1 ||
+      (h->after_previous != 0 && h->after_previous != 1))
     return TILEMIX_ERR_INVALID_ARG;
   const int32_t* cu = h->cu_seqlens_h;
   const int nseq = a->nseq;
@@ -347,15 +348,16 @@ TILEMIX_API int tilemix_prefill_host(const tilemix_prefill_host_args* h, void* s
   cudaStream_t sin = static_cast<cudaStream_t>(h->stream_in);
   cudaStream_t sout = static_cast<cudaStream_t>(h->stream_out);
   cudaEvent_t* ev = static_cast<cudaEvent_t*>(h->events);
-  cudaEvent_t join = ev[2 * h->chunks];
+  cudaEvent_t join = ev[3 * h->chunks];
   const size_t qrow = static_cast<size_t>(a->hq) * a->d * 2;  // bytes per token
   const size_t krow = static_cast<size_t>(a->hk) * a->d * 2;
   auto at = [](const void* base, size_t off) {
     return static_cast<void*>(static_cast<uint8_t*>(const_cast<void*>(base)) + off);
   };
-  // uploads start once `stream` has finished what precedes this call (a
-  // previous call's kernels and downloads use the same device rows)
-  if (cudaEventRecord(join, st) != cudaSuccess || cudaStreamWaitEvent(sin, join, 0) != cudaSuccess)
+  // unless the call follows one on the same rows, uploads start once
+  // `stream` has finished what precedes this call
+  if (!h->after_previous &&
+      (cudaEventRecord(join, st) != cudaSuccess || cudaStreamWaitEvent(sin, join, 0) != cudaSuccess))
     return TILEMIX_ERR_CUDA;
   // run c: whole sequences s0 .. s1 - 1, cut where the token count first
   // reaches (c + 1) / chunks of the batch
@@ -373,21 +375,27 @@ TILEMIX_API int tilemix_prefill_host(const tilemix_prefill_host_args* h, void* s
     }
     const size_t t0 = static_cast<size_t>(cu[s0]), n = static_cast<size_t>(cu[s1]) - t0;
     if (n > 0) {
-      if (cudaMemcpyAsync(at(a->q, t0 * qrow), at(h->q_h, t0 * qrow), n * qrow,
+      // events of run c: upload done, kernels done, download done; waiting on
+      // the last two first orders this run after the previous call's run c
+      cudaEvent_t up = ev[3 * c], kern = ev[3 * c + 1], down = ev[3 * c + 2];
+      if (cudaStreamWaitEvent(sin, kern, 0) != cudaSuccess ||
+          cudaMemcpyAsync(at(a->q, t0 * qrow), at(h->q_h, t0 * qrow), n * qrow,
                           cudaMemcpyHostToDevice, sin) != cudaSuccess ||
           cudaMemcpyAsync(at(a->k, t0 * krow), at(h->k_h, t0 * krow), n * krow,
                           cudaMemcpyHostToDevice, sin) != cudaSuccess ||
           cudaMemcpyAsync(at(a->v, t0 * krow), at(h->v_h, t0 * krow), n * krow,
                           cudaMemcpyHostToDevice, sin) != cudaSuccess ||
-          cudaEventRecord(ev[2 * c], sin) != cudaSuccess ||
-          cudaStreamWaitEvent(st, ev[2 * c], 0) != cudaSuccess)
+          cudaEventRecord(up, sin) != cudaSuccess ||
+          cudaStreamWaitEvent(st, up, 0) != cudaSuccess ||
+          cudaStreamWaitEvent(st, down, 0) != cudaSuccess)
         return TILEMIX_ERR_CUDA;
       rc = run_prefill_range(a, pl, s0, s1, {q0, nqt, k0, nkt}, longest, st);
       if (rc != TILEMIX_OK) return rc;
-      if (cudaEventRecord(ev[2 * c + 1], st) != cudaSuccess ||
-          cudaStreamWaitEvent(sout, ev[2 * c + 1], 0) != cudaSuccess ||
+      if (cudaEventRecord(kern, st) != cudaSuccess ||
+          cudaStreamWaitEvent(sout, kern, 0) != cudaSuccess ||
           cudaMemcpyAsync(at(h->o_h, t0 * qrow), at(a->o, t0 * qrow), n * qrow,
-                          cudaMemcpyDeviceToHost, sout) != cudaSuccess)
+                          cudaMemcpyDeviceToHost, sout) != cudaSuccess ||
+          cudaEventRecord(down, sout) != cudaSuccess)
         return TILEMIX_ERR_CUDA;
     }
     s0 = s1;

@@ -71,10 +71,12 @@ class TileMixPrefill:
         tilemix_prefill_fwd(self.args(q, k, v, o, lse=lse, **kw), stream)
         return o
 
-    def host_args(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8):
+    def host_args(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8, after_previous=False):
         """Arguments of ``tilemix_prefill_host``: host tensors q_h, k_h, v_h, o_h
         (page-locked for the copies to overlap) and the device buffers q, k, v,
-        o of the same shapes.  The side streams and events are kept here."""
+        o of the same shapes.  The side streams and events are kept here, so
+        ``after_previous`` may chain a call to the previous one made through
+        this object with the same device buffers and chunks."""
         for name, t in (("q_h", q_h), ("k_h", k_h), ("v_h", v_h), ("o_h", o_h)):
             if t.device.type != "cpu" or not t.is_contiguous() or t.dtype != torch.float16:
                 raise ValueError("%s must be a contiguous fp16 CPU tensor" % name)
@@ -82,7 +84,7 @@ class TileMixPrefill:
         if self._host_side is None or self._host_side[0] != chunks:
             s_in = torch.cuda.Stream(device=self.device)
             s_out = torch.cuda.Stream(device=self.device)
-            evs = [torch.cuda.Event() for _ in range(2 * chunks + 1)]
+            evs = [torch.cuda.Event() for _ in range(3 * chunks + 1)]
             for e in evs:  # creates the CUDA event
                 e.record(s_in)
             handles = (ctypes.c_void_p * len(evs))(*[e.cuda_event for e in evs])
@@ -97,10 +99,18 @@ class TileMixPrefill:
         h.stream_in = s_in.cuda_stream
         h.stream_out = s_out.cuda_stream
         h.events = ctypes.cast(handles, ctypes.c_void_p).value
+        h.after_previous = 1 if after_previous else 0
         return h
 
-    def from_host(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8, stream=None):
+    @property
+    def upload_stream(self):
+        """The stream the host-buffer call uploads on (None before its first use)."""
+        return None if self._host_side is None else self._host_side[1]
+
+    def from_host(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8, after_previous=False,
+                  stream=None):
         """O of host inputs into host o_h through tilemix_prefill_host; work
         enqueued on `stream` afterwards sees o_h complete."""
-        tilemix_prefill_host(self.host_args(q_h, k_h, v_h, o_h, q, k, v, o, chunks), stream)
+        tilemix_prefill_host(self.host_args(q_h, k_h, v_h, o_h, q, k, v, o, chunks,
+                                            after_previous), stream)
         return o_h
