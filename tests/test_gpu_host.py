@@ -114,3 +114,30 @@ def test_host_prefill_workload_equals_device_call():
     want = gc.run_gpu(case, q, k, v, masks)["o"]
     got = _host_run(case, q, k, v, masks, chunks=8)
     assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+
+
+def test_host_prefill_fp8_lse_and_head_map_equal_device_call():
+    """The FP8 low path, the LSE output (left on the device) and a custom
+    query-to-KV head map go through the host-buffer call unchanged."""
+    import tile_routed_mixed_b200 as tm
+    case = gc.Case([77, 640, 129, 300], 4, 2, 128, template="bigbird", percent=60, seed=5,
+                   kv_map=[1, 0, 0, 1])
+    q, k, v = case.inputs()
+    masks = case.masks()
+    pf = tm.TileMixPrefill(case.lengths, case.hq, case.hk, case.d, masks, case.g,
+                           causal=case.causal, kv_head_of_q=case.kv_map, low="fp8")
+    qd, kd, vd = (torch.from_numpy(x).cuda() for x in (q, k, v))
+    od = torch.empty_like(qd)
+    lse_dev = torch.zeros((case.hq, case.total_tokens), dtype=torch.float32, device="cuda")
+    pf(qd, kd, vd, od, lse=lse_dev)
+    torch.cuda.synchronize()
+    want_o, want_lse = od.cpu().numpy(), lse_dev.cpu().numpy()
+    qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    oh = torch.full(q.shape, float("nan"), dtype=torch.float16).pin_memory()
+    q2, k2, v2, o2 = (torch.empty_like(x) for x in (qd, kd, vd, od))
+    lse2 = torch.zeros_like(lse_dev)
+    pf.from_host(qh, kh, vh, oh, q2, k2, v2, o2, chunks=3, lse=lse2)
+    torch.cuda.current_stream().synchronize()
+    assert tm.tilemix_get_error() == tm.OK
+    assert np.array_equal(oh.numpy().view(np.uint16), want_o.view(np.uint16))
+    assert np.array_equal(lse2.cpu().numpy().view(np.uint32), want_lse.view(np.uint32))

@@ -71,12 +71,14 @@ class TileMixPrefill:
         tilemix_prefill_fwd(self.args(q, k, v, o, lse=lse, **kw), stream)
         return o
 
-    def host_args(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8, after_previous=False):
+    def host_args(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8, after_previous=False,
+                  lse=None):
         """Arguments of ``tilemix_prefill_host``: host tensors q_h, k_h, v_h, o_h
         (page-locked for the copies to overlap) and the device buffers q, k, v,
         o of the same shapes.  The side streams and events are kept here, so
         ``after_previous`` may chain a call to the previous one made through
-        this object with the same device buffers and chunks."""
+        this object with the same device buffers and chunks.  ``lse``, if
+        given, is a device buffer and stays on the device."""
         for name, t in (("q_h", q_h), ("k_h", k_h), ("v_h", v_h), ("o_h", o_h)):
             if t.device.type != "cpu" or not t.is_contiguous() or t.dtype != torch.float16:
                 raise ValueError("%s must be a contiguous fp16 CPU tensor" % name)
@@ -90,9 +92,9 @@ class TileMixPrefill:
             handles = (ctypes.c_void_p * len(evs))(*[e.cuda_event for e in evs])
             self._host_side = (chunks, s_in, s_out, evs, handles)
         _, s_in, s_out, _, handles = self._host_side
-        self.ensure_workspace(q, k, v, o)
+        self.ensure_workspace(q, k, v, o, lse=lse)
         h = PrefillHostArgs()
-        h.dev = self.args(q, k, v, o)
+        h.dev = self.args(q, k, v, o, lse=lse)
         h.cu_seqlens_h = self.cu_host.ctypes.data
         h.q_h, h.k_h, h.v_h, h.o_h = (t.data_ptr() for t in (q_h, k_h, v_h, o_h))
         h.chunks = chunks
@@ -108,9 +110,9 @@ class TileMixPrefill:
         return None if self._host_side is None else self._host_side[1]
 
     def from_host(self, q_h, k_h, v_h, o_h, q, k, v, o, chunks=8, after_previous=False,
-                  stream=None):
+                  lse=None, stream=None):
         """O of host inputs into host o_h through tilemix_prefill_host; work
         enqueued on `stream` afterwards sees o_h complete."""
         tilemix_prefill_host(self.host_args(q_h, k_h, v_h, o_h, q, k, v, o, chunks,
-                                            after_previous), stream)
+                                            after_previous, lse), stream)
         return o_h
