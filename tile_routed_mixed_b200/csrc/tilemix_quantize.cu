@@ -19,12 +19,11 @@ namespace tilemix {
 // Block quantisation ("only Q and K are quantised, Q in 128 x d blocks and K
 // in 64 x d blocks, symmetric absmax / 127").  One launch covers every Q block
 // and every K block; one CTA per (block, head) holds its block in registers
-// (at most eight 16-byte chunks per thread), so HBM sees each fp16 element
-// read once and each code written once.  codes = clamp(rne(x / s), +-127)
-// with s = a / 127, both divisions IEEE fp32.
+// (at most eight 16-byte chunks per thread at d = 128, four at d = 64), so
+// HBM sees each fp16 element read once and each code written once.
+// codes = clamp(rne(x / s), +-127) with s = a / 127, both divisions IEEE fp32.
 // ===================================================================
 constexpr int kQuantThreads = 256;
-constexpr int kQuantChunks = 8;  // per thread: 128 rows x 128 dims / 8 / 256
 
 // One tensor's blocks: tiles tile0 .. tile0 + ntiles - 1 (cu_tiles holds the
 // sequences' first tiles, cu_tiles[0] <= tile0), scales [heads][total_tiles].
@@ -38,9 +37,15 @@ struct QuantSide {
 
 // fp8 != 0: the FP8 low path's codes instead, e4m3(x / s) with s = a / 448
 // (round to nearest even, saturating; IEEE fp32 division for both).
-__global__ void __launch_bounds__(kQuantThreads)
+// Thread t takes the 16-byte chunks of rows t / C + j 256 / C (C chunks per
+// row), column t mod C, for j < kChunks.
+template <int D>
+__global__ void __launch_bounds__(kQuantThreads, D == 128 ? 4 : 5)
     quantize_qk_kernel(QuantSide qs, QuantSide ks, const int32_t* __restrict__ cu_seqlens,
-                       int nseq, int d, int* ticket, int fp8) {
+                       int nseq, int* ticket, int fp8) {
+  constexpr int kCprLog2 = D == 128 ? 4 : 3;                 // 16-byte chunks per row
+  constexpr int kRowsPerPass = kQuantThreads >> kCprLog2;    // rows one pass covers
+  constexpr int kChunks = TILEMIX_BLOCK_M / kRowsPerPass;    // passes over a Q block
   if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;
   const int nq = qs.ntiles * qs.heads;
   const bool is_q = static_cast<int>(blockIdx.x) < nq;
@@ -66,21 +71,21 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int L = __ldg(cu_seqlens + lo + 1) - t0;
   const int r0 = (tile - __ldg(cu_tiles + lo)) * block_rows;
   const int rows = min(block_rows, L - r0);
-  const int cpr_log2 = d == 128 ? 4 : 3;  // 16-byte chunks per row
-  const int nchunks = rows << cpr_log2;
-  const size_t row_stride = static_cast<size_t>(heads) * d;
-  const size_t base = (static_cast<size_t>(t0 + r0) * heads + h) * d;
+  const size_t base = (static_cast<size_t>(t0 + r0) * heads + h) * D;
+  // offsets inside the block fit 32 bits: rows x heads x d <= 128 x 256 x 128
+  const int row_stride = heads * D;
+  const int row0 = threadIdx.x >> kCprLog2;
+  const int off0 = row0 * row_stride + ((threadIdx.x & ((1 << kCprLog2) - 1)) << 3);
+  const int step = kRowsPerPass * row_stride;
+  const __half* xb = x + base;
+  int8_t* cb = codes + base;
 
-  uint4 u[kQuantChunks];
+  uint4 u[kChunks];
   __half2 amax2 = __float2half2_rn(0.f);
 #pragma unroll
-  for (int i = 0; i < kQuantChunks; ++i) {
-    const int c = threadIdx.x + i * kQuantThreads;
+  for (int i = 0; i < kChunks; ++i) {
     u[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (c < nchunks) {
-      const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
-      u[i] = *reinterpret_cast<const uint4*>(x + off);
-    }
+    if (row0 + i * kRowsPerPass < rows) u[i] = *reinterpret_cast<const uint4*>(xb + off0 + i * step);
     const __half2* hv = reinterpret_cast<const __half2*>(&u[i]);
 #pragma unroll
     for (int k = 0; k < 4; ++k) amax2 = __hmax2(amax2, __habs2(hv[k]));
@@ -99,9 +104,8 @@ __global__ void __launch_bounds__(kQuantThreads)
   const float r = a > 0.f ? __frcp_rn(s) : 0.f;
   if (fp8) {
 #pragma unroll
-    for (int i = 0; i < kQuantChunks; ++i) {
-      const int c = threadIdx.x + i * kQuantThreads;
-      if (c < nchunks) {
+    for (int i = 0; i < kChunks; ++i) {
+      if (row0 + i * kRowsPerPass < rows) {
         uint32_t w[2] = {0u, 0u};
         if (a > 0.f) {
           const __half* hv = reinterpret_cast<const __half*>(&u[i]);
@@ -112,20 +116,17 @@ __global__ void __launch_bounds__(kQuantThreads)
             w[e >> 2] |= b8 << (8 * (e & 3));
           }
         }
-        const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
-        *reinterpret_cast<uint2*>(codes + off) = make_uint2(w[0], w[1]);
+        *reinterpret_cast<uint2*>(cb + off0 + i * step) = make_uint2(w[0], w[1]);
       }
     }
     return;
   }
 
 #pragma unroll
-  for (int i = 0; i < kQuantChunks; ++i) {
-    const int c = threadIdx.x + i * kQuantThreads;
-    if (c < nchunks) {
+  for (int i = 0; i < kChunks; ++i) {
+    if (row0 + i * kRowsPerPass < rows) {
       const uint2 packed = a > 0.f ? quant_chunk(u[i], s, r) : make_uint2(0u, 0u);
-      const size_t off = base + (c >> cpr_log2) * row_stride + ((c & ((1 << cpr_log2) - 1)) << 3);
-      *reinterpret_cast<uint2*>(codes + off) = packed;
+      *reinterpret_cast<uint2*>(cb + off0 + i * step) = packed;
     }
   }
 }
@@ -144,8 +145,12 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
   if (blocks == 0)
     return ticket ? static_cast<int>(cudaMemsetAsync(ticket, 0, sizeof(int), stream)) : cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  quantize_qk_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-      qs, ks, cu_seqlens, nseq, d, ticket, fp8);
+  if (d == 128)
+    quantize_qk_kernel<128><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+        qs, ks, cu_seqlens, nseq, ticket, fp8);
+  else
+    quantize_qk_kernel<64><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+        qs, ks, cu_seqlens, nseq, ticket, fp8);
   return static_cast<int>(cudaGetLastError());
 }
 
