@@ -243,6 +243,25 @@ __device__ __forceinline__ void add_f16x2_to_f32(float& s, uint32_t h2) {
       : "r"(h2));
 }
 
+// {a0 * b + c, a1 * b + c} as one packed instruction (sm_100 fp32x2; each
+// lane is the IEEE fused multiply-add fmaf gives); b2 and c2 hold b and c in
+// both lanes.
+__device__ __forceinline__ float2 fma2_bc(float a0, float a1, unsigned long long b2,
+                                          unsigned long long c2) {
+  unsigned long long a, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b2), "l"(c2));
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long both_lanes(float x) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -445,11 +464,11 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st,
   const float alpha = resc ? ptx::ex2(st.m - m_new) : 1.0f;
   float ls[4] = {0.f, 0.f, 0.f, 0.f};
   // P = 2^(score * c - m), packed in place: pair k lands in r[k]
+  const unsigned long long c2 = both_lanes(c), nm2 = both_lanes(-m_use);
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
-    const float x0 = fmaf(__uint_as_float(r[2 * k]), c, -m_use);
-    const float x1 = fmaf(__uint_as_float(r[2 * k + 1]), c, -m_use);
-    r[k] = pack_f16x2(ptx::ex2(x0), ptx::ex2(x1));
+    const float2 x = fma2_bc(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]), c2, nm2);
+    r[k] = pack_f16x2(ptx::ex2(x.x), ptx::ex2(x.y));
     add_f16x2_to_f32(ls[k & 3], r[k]);
   }
   if (masked && c == 0.f) {
