@@ -90,6 +90,17 @@ int tilemix_auto_g(int seqlen, int* g_out);
 int tilemix_tile_offsets(const int32_t* cu_seqlens_h, int nseq, int32_t* cu_qtiles_h,
                          int32_t* cu_ktiles_h);
 
+/* The runs of whole sequences tilemix_prefill_host cuts a batch into:
+ * run r holds sequences run_start_h[r] .. run_start_h[r + 1] - 1, r < *nruns.
+ * Run c ends before the first sequence s whose token offset cu_seqlens_h[s]
+ * reaches (c + 1) / min(chunks, nseq) of the batch's tokens; the last run
+ * takes every remaining sequence.  run_start_h: host, min(chunks, nseq) + 1
+ * entries, caller-allocated (run_start_h[0] = 0, run_start_h[*nruns] = nseq).
+ * INVALID_ARG on NULL pointers, nseq < 0, chunks < 1 or offsets that do not
+ * start at 0 or decrease. */
+int tilemix_host_runs(const int32_t* cu_seqlens_h, int nseq, int chunks, int32_t* run_start_h,
+                      int* nruns);
+
 /* Routing words of a static template at a stated INT8 coverage of legal tile
  * groups (TileMix pages: data-free templates borrowed from sparse attention;
  * coverage is the share of legal groups routed INT8, not a FLOP share; the

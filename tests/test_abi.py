@@ -194,6 +194,56 @@ def test_prefill_host_argument_checks_are_synchronous():
     assert L.tilemix_prefill_host(ctypes.byref(host(dev_nseq=0)), None) == tm.OK
 
 
+def _runs_reference(lengths, chunks):
+    """The host-buffer call's cut rule restated: with n = min(chunks, nseq),
+    run c ends before the first sequence whose start offset reaches
+    (c + 1) / n of the tokens; the last run takes the rest."""
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    nseq = len(lengths)
+    n = min(chunks, nseq)
+    starts, s0 = [0], 0
+    for c in range(n):
+        if s0 >= nseq:
+            break
+        s1 = s0 + 1
+        while s1 < nseq and (c == n - 1 or cu[s1] < cu[-1] * (c + 1) // n):
+            s1 += 1
+        starts.append(s1)
+        s0 = s1
+    return starts
+
+
+@pytest.mark.parametrize("lengths,chunks", [
+    ([4096] * 8, 8), ([4096] * 8, 3), ([4096] * 8, 16), ([100, 1, 3000, 7, 7, 512], 4),
+    ([5000, 10, 10, 10], 2), ([1], 5), ([0, 0, 64, 0], 3), ([300, 1, 777, 128, 197], 3),
+])
+def test_host_runs_cut_rule(lengths, chunks):
+    starts = tm.tilemix_host_runs(np.concatenate([[0], np.cumsum(lengths)]), chunks)
+    assert list(starts) == _runs_reference(lengths, chunks)
+    # every sequence in exactly one run, in order, no empty run
+    assert starts[0] == 0 and starts[-1] == len(lengths)
+    assert all(b > a for a, b in zip(starts[:-1], starts[1:]))
+    assert len(starts) - 1 <= min(chunks, len(lengths))
+
+
+def test_host_runs_equal_sequences_split_evenly():
+    starts = tm.tilemix_host_runs(np.arange(0, 8 * 4096 + 1, 4096), 4)
+    assert list(starts) == [0, 2, 4, 6, 8]
+
+
+def test_host_runs_rejects_bad_arguments():
+    L = tm.lib()
+    cu = np.array([0, 10, 5], dtype=np.int32)   # decreasing
+    out = np.zeros(4, dtype=np.int32)
+    n = ctypes.c_int(0)
+    assert L.tilemix_host_runs(cu.ctypes.data, 2, 2, out.ctypes.data, ctypes.byref(n)) == \
+        tm.ERR_INVALID_ARG
+    ok = np.array([0, 10, 15], dtype=np.int32)
+    assert L.tilemix_host_runs(ok.ctypes.data, 2, 0, out.ctypes.data, ctypes.byref(n)) == \
+        tm.ERR_INVALID_ARG
+    assert L.tilemix_host_runs(None, 2, 2, out.ctypes.data, ctypes.byref(n)) == tm.ERR_INVALID_ARG
+
+
 def _fake_decode(**over):
     a = tm.DecodeArgs()
     for f in ("q", "k", "v", "k_i8", "k_scale", "o", "seq_start", "seq_len", "ktile_start",

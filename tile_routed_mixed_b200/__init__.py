@@ -134,6 +134,8 @@ def lib():
         L.tilemix_auto_g.argtypes = [I, P]
         L.tilemix_tile_offsets.restype = I
         L.tilemix_tile_offsets.argtypes = [P, I, P, P]
+        L.tilemix_host_runs.restype = I
+        L.tilemix_host_runs.argtypes = [P, I, I, P, P]
         L.tilemix_build_routing.restype = I
         L.tilemix_build_routing.argtypes = [I, I, ctypes.c_uint64, P, I, I, P, I, P, P, P]
         L.tilemix_quantize_qk.restype = I
@@ -212,6 +214,18 @@ def tilemix_tile_offsets(cu_seqlens):
     _check(lib().tilemix_tile_offsets(cu.ctypes.data, nseq, cq.ctypes.data, ck.ctypes.data),
            "tilemix_tile_offsets")
     return cq, ck
+
+
+def tilemix_host_runs(cu_seqlens, chunks: int):
+    """First sequence of each run tilemix_prefill_host cuts the batch into,
+    plus nseq at the end (so run r is run_start[r] .. run_start[r + 1] - 1)."""
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    nseq = cu.size - 1
+    starts = np.zeros(max(1, min(int(chunks), nseq)) + 1, dtype=np.int32)
+    n = ctypes.c_int(0)
+    _check(lib().tilemix_host_runs(cu.ctypes.data, nseq, int(chunks), starts.ctypes.data,
+                                   ctypes.byref(n)), "tilemix_host_runs")
+    return starts[:n.value + 1].copy()
 
 
 def tilemix_build_routing(template, int8_percent: int, seed: int, cu_seqlens, n_kv_heads: int,
@@ -447,7 +461,7 @@ __all__ = [
     "tilemix_build_routing", "tilemix_decode_fwd", "tilemix_decode_workspace_size",
     "tilemix_get_error", "tilemix_prefill_fwd",
     "tilemix_prefill_fwd_noalloc", "tilemix_quantize_qk", "tilemix_selftest_wait_timeout",
-    "PrefillHostArgs", "tilemix_prefill_host",
+    "PrefillHostArgs", "tilemix_prefill_host", "tilemix_host_runs",
     "tilemix_status_string", "tilemix_tile_offsets", "tilemix_version",
     "tilemix_workspace_size",
 ]

@@ -363,9 +363,7 @@ TILEMIX_API int tilemix_prefill_host(const tilemix_prefill_host_args* h, void* s
   // reaches (c + 1) / chunks of the batch
   int s0 = 0, q0 = 0, k0 = 0;
   for (int c = 0; c < chunks && s0 < nseq; ++c) {
-    const long long target = static_cast<long long>(a->total_tokens) * (c + 1) / chunks;
-    int s1 = s0 + 1;
-    while (s1 < nseq && (c == chunks - 1 || cu[s1] < target)) ++s1;
+    const int s1 = tilemix::run_end(cu, nseq, chunks, c, s0);
     int nqt = 0, nkt = 0, longest = 0;
     for (int s = s0; s < s1; ++s) {
       const int L = cu[s + 1] - cu[s];

@@ -162,6 +162,24 @@ TILEMIX_API int tilemix_auto_g(int seqlen, int* g_out) {
   return TILEMIX_OK;
 }
 
+TILEMIX_API int tilemix_host_runs(const int32_t* cu_seqlens_h, int nseq, int chunks,
+                                  int32_t* run_start_h, int* nruns) {
+  if (!cu_seqlens_h || !run_start_h || !nruns || nseq < 0 || chunks < 1)
+    return TILEMIX_ERR_INVALID_ARG;
+  if (cu_seqlens_h[0] != 0) return TILEMIX_ERR_INVALID_ARG;
+  for (int s = 0; s < nseq; ++s)
+    if (cu_seqlens_h[s + 1] < cu_seqlens_h[s]) return TILEMIX_ERR_INVALID_ARG;
+  const int n = chunks < nseq ? chunks : nseq;
+  int r = 0, s0 = 0;
+  run_start_h[0] = 0;
+  for (int c = 0; c < n && s0 < nseq; ++c) {
+    s0 = tilemix::run_end(cu_seqlens_h, nseq, n, c, s0);
+    run_start_h[++r] = s0;
+  }
+  *nruns = r;
+  return TILEMIX_OK;
+}
+
 TILEMIX_API int tilemix_tile_offsets(const int32_t* cu_seqlens_h, int nseq, int32_t* cu_qtiles_h,
                                      int32_t* cu_ktiles_h) {
   if (!cu_seqlens_h || !cu_qtiles_h || !cu_ktiles_h || nseq < 0) return TILEMIX_ERR_INVALID_ARG;

@@ -111,6 +111,17 @@ int launch_decode(const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_beg
 // One launch quantises Q (128-row blocks) and K (64-row blocks); a null q or
 // k skips that side.  A non-null ticket is set to zero by the same launch
 // (the fused kernel that follows on the stream hands out work from it).
+// Runs of whole sequences for the host-buffer prefill: run c (c < chunks)
+// starts at sequence s0 and ends before the returned s1, the first s > s0
+// whose token offset cu[s] reaches (c + 1) / chunks of the batch (the last
+// run takes every remaining sequence).  Host code; cu has nseq + 1 entries.
+inline int run_end(const int32_t* cu, int nseq, int chunks, int c, int s0) {
+  const long long target = static_cast<long long>(cu[nseq]) * (c + 1) / chunks;
+  int s1 = s0 + 1;
+  while (s1 < nseq && (c == chunks - 1 || cu[s1] < target)) ++s1;
+  return s1;
+}
+
 // Tiles a quantisation launch covers: Q tiles qtile0 .. qtile0 + nqtiles - 1
 // and K tiles ktile0 .. ktile0 + nktiles - 1, those of the nseq sequences
 // whose offsets cu_seqlens / cu_qtiles / cu_ktiles point at (a whole batch, or
