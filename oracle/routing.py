@@ -103,7 +103,7 @@ def int8_target(percent: int, N: int) -> int:
 def _fixed_width(n, F):
     """Per-row FP16 counts of the fixed-width rule (Band / Global)."""
     w = 0
-    while w < max(n) and sum(min(w + 1, x) for x in n) <= F:
+    while n and w < max(n) and sum(min(w + 1, x) for x in n) <= F:
         w += 1
     left = F - sum(min(w, x) for x in n)
     widths = []

@@ -57,6 +57,9 @@ def _geometries():
     out.append(("ragged", [100, 300, 1, 513, 2000], [1, 1, 1, 1, 1], True))
     out.append(("ragged_noncausal", [100, 300, 513], [1, 1, 1], False))
     out.append(("g3", [5000, 3000], [3, 2], True))
+    # zero-length sequences have no query-tile rows and so no words
+    out.append(("empty_seqs", [0, 300, 0, 64, 0], [1, 1, 1, 1, 1], True))
+    out.append(("only_empty", [0, 0], [1, 1], True))
     return out
 
 
