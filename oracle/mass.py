@@ -50,6 +50,8 @@ def probe_rows(q16, k16, masks, g, lengths, causal, delta=4.0, kv_map=None, band
     start = 0
     cq = 0
     for s, L in enumerate(lengths):
+        if L == 0:  # no rows, nothing to write
+            continue
         gs = int(g[s])
         for h in range(hq):
             kv = h // (hq // hk) if kv_map is None else int(kv_map[h])

@@ -667,6 +667,27 @@ def test_mass_probe_all_fp16_and_all_int8_words():
     assert np.all(r1["h"] <= 1 + 1e-12) and np.all(r1["h"] > 0)
 
 
+def test_empty_sequences_change_nothing():
+    """Zero-length sequences hold no rows and no tiles: a batch with them
+    inserted gives the same mass-probe rows and adaptive words as without."""
+    rng = np.random.default_rng(5)
+    hq, hk, d = 2, 1, 64
+    q = rng.standard_normal((194, hq, d)).astype(np.float16)
+    k = rng.standard_normal((194, hk, d)).astype(np.float16)
+    plain, padded = [130, 64], [0, 130, 0, 64, 0]
+    g_plain, g_padded = [1, 1], [1, 1, 1, 1, 1]
+    m_plain = oracle.build_routing("sptrans", 75, 0, plain, hk, g_plain, True)[0]
+    m_padded = oracle.build_routing("sptrans", 75, 0, padded, hk, g_padded, True)[0]
+    assert np.array_equal(m_plain, m_padded)
+    a = om.probe_rows(q, k, m_plain, g_plain, plain, True)
+    b = om.probe_rows(q, k, m_padded, g_padded, padded, True)
+    for key in a:
+        assert np.array_equal(a[key], b[key]), key
+    w_plain = ad.route_pooled(q, k, plain, hq, hk, g_plain, True, 50)
+    w_padded = ad.route_pooled(q, k, padded, hq, hk, g_padded, True, 50)
+    assert np.array_equal(w_plain, w_padded)
+
+
 def test_mass_probe_uniform_scores_closed_form():
     # q = 0: every legal key scores 0, P is uniform over the i + 1 legal keys,
     # every key is high-importance, and the INT8 mass is the INT8 key count
