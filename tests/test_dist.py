@@ -44,3 +44,23 @@ def test_single_process_is_identity():
     import bench
     assert bench.max_over_ranks([3.5, 1.25]) == [3.5, 1.25]
     assert bench.whole_job_tokens(32768, 1) == 32768
+
+
+def test_reference_arm_under_torchrun_two_ranks(root):
+    """`bench.py --impl reference` launched as the driver launches N > 1: rank
+    0 alone times the oracle and prints one JSON line, the other rank exits 0
+    without work."""
+    import json
+    import subprocess
+    import sys
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "2", "--warmup", "3", "--workload", "tiny_l256"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["config"]["workload"] == "tiny_l256"
