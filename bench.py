@@ -194,11 +194,23 @@ def kernel_traffic(workload_name, kernel="prefill_fwd_kernel<128>"):
         return None
 
 
-def host_cores():
+def affinity_cores():
     try:
         return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count() or 1
+
+
+def host_cores():
+    """Threads the oracle's OpenMP loops run on: OMP_NUM_THREADS when set,
+    else every core this process may use."""
+    try:
+        n = int(os.environ.get("OMP_NUM_THREADS", "").split(",")[0])
+        if n > 0:
+            return n
+    except ValueError:
+        pass
+    return affinity_cores()
 
 
 # ------------------------------------------------------------ oracle side ---
@@ -248,6 +260,11 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        # the launcher pins every rank to one OpenMP thread; rank 0 works
+        # alone here, so give the oracle every core (before any OpenMP
+        # runtime loads)
+        os.environ["OMP_NUM_THREADS"] = str(affinity_cores())
     w, lengths, g = workload(args.workload, args.template, args.percent)
     hq, hk, d, causal = w["hq"], w["hk"], w["d"], w["causal"]
     T = sum(lengths)

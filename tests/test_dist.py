@@ -64,3 +64,5 @@ def test_reference_arm_under_torchrun_two_ranks(root):
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["config"]["workload"] == "tiny_l256"
+    # rank 0 gives the oracle every core even though the launcher pins one thread
+    assert line["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
