@@ -268,7 +268,8 @@ int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
  *   k_h, v_h      host fp16 [total_tokens][hk][d] ...
  *   o_h           host fp16 [total_tokens][hq][d] (output); the copies only
  *                 overlap anything when these four are page-locked memory
- *   chunks        >= 1, the most runs to cut the batch into (at most nseq)
+ *   chunks        1 .. 2^20, the most runs to cut the batch into (at most
+ *                 nseq are made)
  *   stream_in, stream_out   two cudaStream_t, each different from `stream`
  *   events        3 * chunks + 1 cudaEvent_t created by the caller (timing
  *                 may be disabled), used by nothing else: per run, its
@@ -284,10 +285,10 @@ int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
  *                 (Run c's waits on events 3c + 1 and 3c + 2 are made in
  *                 both modes; an event never recorded is no wait.)
  * INVALID_ARG also when a host pointer, a stream or `events` is NULL, chunks
- * < 1, after_previous not 0 or 1, or cu_seqlens_h disagrees with total_tokens, total_qtiles,
- * total_ktiles or max_seqlen (all checked before anything is enqueued);
- * otherwise as tilemix_prefill_fwd.  On CUDA, part of the work may already
- * be enqueued. */
+ * is outside 1 .. 2^20, after_previous is not 0 or 1, or cu_seqlens_h
+ * disagrees with total_tokens, total_qtiles, total_ktiles or max_seqlen (all
+ * checked before anything is enqueued); otherwise as tilemix_prefill_fwd.
+ * On CUDA, part of the work may already be enqueued. */
 typedef struct tilemix_prefill_host_args {
   tilemix_prefill_args dev;
   const int32_t* cu_seqlens_h;

@@ -180,6 +180,7 @@ def test_prefill_host_argument_checks_are_synchronous():
         (dict(stream_in=None), tm.ERR_INVALID_ARG),
         (dict(events=None), tm.ERR_INVALID_ARG),
         (dict(chunks=0), tm.ERR_INVALID_ARG),
+        (dict(chunks=(1 << 20) + 1), tm.ERR_INVALID_ARG),  # 3 * chunks + 1 events must fit
         (dict(after_previous=2), tm.ERR_INVALID_ARG),
         (dict(cu_seqlens_h=None), tm.ERR_INVALID_ARG),
         (dict(dev_total_qtiles=4), tm.ERR_INVALID_ARG),  # disagrees with the host offsets

@@ -325,7 +325,7 @@ TILEMIX_API int tilemix_prefill_host(const tilemix_prefill_host_args* h, void* s
   if (rc != TILEMIX_OK) return rc;
   if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;
   if (!h->cu_seqlens_h || !h->q_h || !h->k_h || !h->v_h || !h->o_h || !h->stream_in ||
-      !h->stream_out || !h->events || h->chunks < 1 ||
+      !h->stream_out || !h->events || h->chunks < 1 || h->chunks > (1 << 20) ||
       (h->after_previous != 0 && h->after_previous != 1))
     return TILEMIX_ERR_INVALID_ARG;
   const int32_t* cu = h->cu_seqlens_h;
