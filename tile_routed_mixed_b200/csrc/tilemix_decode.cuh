@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
   const int ktile0 = __ldg(p.ktile_start + s);
   const uint64_t word =
       __ldg(p.masks + static_cast<size_t>(__ldg(p.qtile_start + s) + t / TILEMIX_BLOCK_M) * p.hk + kv);
-  const bool bad = (ntiles - 1) / gs > 63;
+  const bool bad = gs < 1 || (ntiles - 1) / gs > 63;  // no division below when bad
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q4 = lane & 3;  // m16n8 fragment: row g (and g + 8), column pair q4
 
