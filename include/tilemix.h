@@ -174,7 +174,8 @@ typedef struct tilemix_prefill_args {
   int total_ktiles;       /* cu_ktiles[nseq] */
   int max_seqlen;         /* max L_s (upper bound accepted) */
   int hq, hk, d;          /* hq % hk == 0; d in {64, 128} */
-  const int32_t* kv_head_of_q; /* device [hq], or NULL for h / (hq / hk) */
+  const int32_t* kv_head_of_q; /* device [hq], or NULL for h / (hq / hk); entries must
+                                  lie in [0, hk) (not checked on the device) */
   const uint64_t* masks;  /* device [total_qtiles][hk] routing words */
   const int32_t* g;       /* device [nseq] grouping factors */
   int causal;             /* 1: key j legal for query i iff j <= i (and j < L_s) */
@@ -352,7 +353,8 @@ typedef struct tilemix_decode_args {
   const int32_t* qtile_start; /* device [nseq]: masks row of each sequence's first query tile */
   const uint64_t* masks;      /* device [total_qtiles][hk] routing words */
   const int32_t* g;           /* device [nseq] routing-group factors */
-  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk) */
+  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk); a query head whose
+                                 entry is outside [0, hk) is not computed */
   int nseq;                   /* >= 0 (0: nothing to do) */
   int max_seqlen;             /* >= every seq_len[s] (sizes the split of the key range) */
   int total_ktiles;           /* columns of k_scale */
@@ -416,7 +418,8 @@ typedef struct tilemix_route_args {
   const int32_t* cu_qtiles;   /* ... and the tile offsets (tilemix_tile_offsets) */
   const int32_t* cu_ktiles;
   const int32_t* g;
-  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk) */
+  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk); an entry outside
+                                 [0, hk) leaves its head out of every mean */
   int nseq, hq, hk, d;        /* d in {64, 128}; at most 256 query heads per KV head */
   int causal;                 /* 0 or 1 */
   int int8_percent;           /* 0..100 */
@@ -466,7 +469,8 @@ typedef struct tilemix_mass_args {
   const int32_t* cu_ktiles;
   const int32_t* g;
   const uint64_t* masks;      /* device [total_qtiles][hk] routing words */
-  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk) */
+  const int32_t* kv_head_of_q;/* device [hq] or NULL => h / (hq / hk); a head whose
+                                 entry is outside [0, hk) is skipped (rows not written) */
   int nseq, hq, hk, d;        /* d in {64, 128} */
   int causal;                 /* 0 or 1 */
   float softmax_scale;        /* 0 => 1 / sqrt(d) */

@@ -60,6 +60,7 @@ __global__ void __launch_bounds__(kMassThreads) mass_probe_kernel(MassParams p) 
   const int start = __ldg(p.cu_seqlens + s);
   const int i0 = (blk - __ldg(p.cu_ktiles + s)) * kMassRows;
   const int kv = p.kv_head_of_q ? __ldg(p.kv_head_of_q + h) : h / (p.hq / p.hk);
+  if (kv < 0 || kv >= p.hk) return;  // a head map entry out of range: the head is skipped
   const uint64_t word =
       __ldg(p.masks + static_cast<size_t>(__ldg(p.cu_qtiles + s) + i0 / TILEMIX_BLOCK_M) * p.hk + kv);
   const int gs = __ldg(p.g + s);
