@@ -383,3 +383,22 @@ def test_mass_probe_argument_checks_are_synchronous():
     a.cu_seqlens_h = empty.ctypes.data_as(ctypes.c_void_p)
     a.g_h = one.ctypes.data_as(ctypes.c_void_p)
     assert L.tilemix_mass_probe(ctypes.byref(a), None) == tm.OK                # nothing to do
+
+
+def test_plain_c_program_against_the_header(tmp_path):
+    """tests/abi_check.c, compiled as C99 with gcc against include/tilemix.h and
+    linked to the library: the ABI needs no Python and no C++ on the caller's
+    side (host entry points and argument checks only; no GPU is touched)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(tm.LIB_PATH)
+    exe = str(tmp_path / "abi_check")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-O1",
+                           "-I" + os.path.join(root, "include"),
+                           os.path.join(root, "tests", "abi_check.c"), "-L" + libdir, "-ltilemix",
+                           "-Wl,-rpath," + libdir, "-o", exe])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
