@@ -25,8 +25,11 @@ explainer (steps one to three).
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py`` against
 brute force, closed forms, hand-derived words and invariants the pages fix.
-The fp16 output values themselves have no printed worked example on the pages:
-beyond those invariants, output-value parity is unpinned.
+The attention outputs are pinned by an independent whole-matrix fp64 brute
+force (``tests/bruteforce.py``: plain softmax attention for all-FP16 words, the
+routed scores key by key for mixed and all-INT8 words) on small batches.  The
+pages print no worked numeric example of an output, so no stored expected
+output value comes from the pages.
 """
 from . import adaptive, fp8, mass
 from .attention import all_rows, attention_rows, build, half_to_double, int_scores
