@@ -174,8 +174,10 @@ typedef struct tilemix_prefill_args {
   int total_ktiles;       /* cu_ktiles[nseq] */
   int max_seqlen;         /* max L_s (upper bound accepted) */
   int hq, hk, d;          /* hq % hk == 0; d in {64, 128} */
-  const int32_t* kv_head_of_q; /* device [hq], or NULL for h / (hq / hk); entries must
-                                  lie in [0, hk) (not checked on the device) */
+  const int32_t* kv_head_of_q; /* device [hq], or NULL for h / (hq / hk); a query head
+                                  whose entry lies outside [0, hk) is skipped (its
+                                  outputs are not written) and tilemix_get_error()
+                                  then reports INVALID_ARG */
   const uint64_t* masks;  /* device [total_qtiles][hk] routing words */
   const int32_t* g;       /* device [nseq] grouping factors */
   int causal;             /* 1: key j legal for query i iff j <= i (and j < L_s) */
@@ -231,12 +233,15 @@ int tilemix_prefill_fwd(const tilemix_prefill_args* args, void* stream);
  * it (tilemix_workspace_size() > 64 MiB) returns TILEMIX_ERR_TOO_LARGE and
  * launches nothing.  Results equal those of tilemix_prefill_fwd.
  *
- * The first call on a device looks up the scratch array's device address
- * (once per device, with that device current); make that first call before
- * any stream capture.  All calls share the one array: calls that overlap on
- * the GPU (on different streams, or from different threads) race on it and
- * must be serialised by the caller.  Nothing in the array needs to start at
- * zero; every call rewrites what it reads. */
+ * The first call in a CUDA context (a device's primary context, with that
+ * device current, or a context the caller made current) looks up the scratch
+ * array's device address in that context; make that first call before any
+ * stream capture.  A context created later, for example after
+ * cudaDeviceReset, gets a lookup of its own on its first call.  All calls
+ * share the one array: calls that overlap on the GPU (on different streams,
+ * or from different threads) race on it and must be serialised by the
+ * caller.  Nothing in the array needs to start at zero; every call rewrites
+ * what it reads. */
 #define TILEMIX_NOALLOC_SCRATCH_BYTES (64u << 20)
 int tilemix_prefill_fwd_noalloc(const tilemix_prefill_args* args, void* stream);
 
@@ -495,9 +500,26 @@ int tilemix_mass_probe(const tilemix_mass_args* args, void* stream);
  * CUDA context stays usable.  INVALID_ARG for an out-of-range timeout. */
 int tilemix_selftest_wait_timeout(int timeout_ms, void* stream);
 
+/* Diagnostic (not a step of the method): the tensor-core rate of the MMA
+ * forms the fused prefill kernel issues, measured on this GPU.  Launches
+ * `ctas` CTAs (1..4096); in each, one thread issues 4 * iters (iters
+ * 1..2^20) back-to-back tcgen05.mma of one form with M = 128 and N = n
+ * (64, 128 or 256) into TMEM, all accumulating into one tile:
+ *   form 0  kind::f16,    A and B in shared memory, K = 16 per MMA
+ *   form 1  kind::i8,     A and B in shared memory, K = 32 per MMA
+ *   form 2  kind::f16,    A in TMEM, B MN-major in shared memory (the P.V form)
+ *   form 3  kind::f8f6f4 (e4m3), A and B in shared memory, K = 32 per MMA
+ * cycles_dev (device, caller-owned, [2 * ctas] int64) receives per CTA the SM
+ * cycles to issue every MMA and the cycles until all completed (-1 if the
+ * completion wait gave up after 2 s).  Operand values are arbitrary small
+ * codes.  Asynchronous on `stream`; INVALID_ARG for an argument out of range,
+ * CUDA if the launch fails. */
+int tilemix_mma_rate(int form, int n, int iters, int ctas, long long* cycles_dev, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word:
  * OK, TIMEOUT (a bounded wait expired), INVALID_ARG (a row needed more than 64
- * groups, or a bad routing-group factor), or CUDA for a sticky CUDA error. */
+ * groups, a bad routing-group factor, or a head-map entry outside [0, hk): the
+ * work items concerned are skipped), or CUDA for a sticky CUDA error. */
 int tilemix_get_error(void* stream);
 
 #ifdef __cplusplus

@@ -151,6 +151,8 @@ def lib():
         L.tilemix_prefill_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), P]
         L.tilemix_prefill_host.restype = I
         L.tilemix_prefill_host.argtypes = [ctypes.POINTER(PrefillHostArgs), P]
+        L.tilemix_mma_rate.restype = I
+        L.tilemix_mma_rate.argtypes = [I, I, I, I, P, P]
         L.tilemix_decode_workspace_size.restype = I
         L.tilemix_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs),
                                                     ctypes.POINTER(ctypes.c_size_t)]
@@ -335,6 +337,47 @@ def tilemix_prefill_host(args: PrefillHostArgs, stream=None):
            "tilemix_prefill_host")
 
 
+MMA_FORMS = {"f16": 0, "i8": 1, "f16_tmem_a": 2, "f8": 3}
+
+
+def tilemix_mma_rate(form, n, iters, ctas, cycles, stream=None):
+    """Diagnostic: back-to-back tcgen05.mma of one form (see include/tilemix.h);
+    ``cycles`` is a device int64 tensor of 2 * ctas (issue, completion cycles
+    per CTA)."""
+    _check(lib().tilemix_mma_rate(MMA_FORMS[form] if isinstance(form, str) else int(form),
+                                  int(n), int(iters), int(ctas), _ptr(cycles),
+                                  _stream_handle(stream)), "tilemix_mma_rate")
+
+
+def mma_rate(form, n, iters=4096, ctas=None, device="cuda"):
+    """Measured rate of one MMA form on every SM: returns a dict with the SM
+    cycles per MMA (issue and completion, median over CTAs), the wall time and
+    the dense rate in TFLOP/s (TOP/s for INT8) over all CTAs.  M = 128, K = 16
+    (f16) or 32 (i8, f8) per MMA."""
+    import torch
+    dev = torch.device(device)
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    cyc = torch.zeros(2 * ctas, dtype=torch.int64, device=dev)
+    tilemix_mma_rate(form, n, 16, ctas, cyc)  # warm-up (module load, clocks)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    tilemix_mma_rate(form, n, iters, ctas, cyc)
+    b.record()
+    torch.cuda.synchronize(dev)
+    c = cyc.cpu().numpy().reshape(ctas, 2)
+    if (c[:, 1] < 0).any():
+        raise TileMixError(ERR_TIMEOUT, "tilemix_mma_rate")
+    nmma = 4 * iters
+    k = 16 if (form in ("f16", "f16_tmem_a", 0, 2)) else 32
+    ms = a.elapsed_time(b)
+    ops = 2.0 * 128 * n * k * nmma * ctas
+    return {"form": form, "n": int(n), "issue_cycles_per_mma": float(np.median(c[:, 0])) / nmma,
+            "cycles_per_mma": float(np.median(c[:, 1])) / nmma, "ms": ms,
+            "tera_ops_per_s": ops / (ms * 1e-3) / 1e12, "ctas": int(ctas)}
+
+
 def tilemix_selftest_wait_timeout(timeout_ms: int, stream=None):
     _check(lib().tilemix_selftest_wait_timeout(int(timeout_ms), _stream_handle(stream)),
            "tilemix_selftest_wait_timeout")
@@ -463,5 +506,5 @@ __all__ = [
     "tilemix_prefill_fwd_noalloc", "tilemix_quantize_qk", "tilemix_selftest_wait_timeout",
     "PrefillHostArgs", "tilemix_prefill_host", "tilemix_host_runs",
     "tilemix_status_string", "tilemix_tile_offsets", "tilemix_version",
-    "tilemix_workspace_size",
+    "tilemix_workspace_size", "tilemix_mma_rate", "mma_rate",
 ]

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtilemix.so")
 SOURCES = ["tilemix_kernels.cu", "tilemix_quantize.cu", "tilemix_route.cu", "tilemix_mass.cu",
-           "api.cpp", "routing.cpp"]
+           "tilemix_mmarate.cu", "api.cpp", "routing.cpp"]
 HEADERS = ["tilemix_internal.h", "tilemix_ptx.cuh", "tilemix_quant.cuh", "tilemix_decode.cuh",
            "tilemix_mma.cuh"]
 NVCC_FLAGS = [

@@ -704,7 +704,8 @@ TILEMIX_API int tilemix_get_error(void* stream) {
   if (tilemix::read_and_clear_status(&status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return TILEMIX_ERR_CUDA;
   if (status & tilemix::kStatusTimeout) return TILEMIX_ERR_TIMEOUT;
-  if (status & tilemix::kStatusBadGroups) return TILEMIX_ERR_INVALID_ARG;
+  if (status & (tilemix::kStatusBadGroups | tilemix::kStatusBadHeadMap))
+    return TILEMIX_ERR_INVALID_ARG;
   return TILEMIX_OK;
 }
 

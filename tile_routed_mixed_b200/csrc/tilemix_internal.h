@@ -14,15 +14,17 @@ namespace tilemix {
 enum : unsigned int {
   kStatusTimeout = 1u,       // a bounded mbarrier wait expired
   kStatusBadGroups = 2u,     // a row needed a routing group index above 63
+  kStatusBadHeadMap = 4u,    // a head-map entry outside [0, hk)
 };
+
 
 // Everything the fused attention kernel needs, by value (kernel parameter).
 struct PrefillParams {
   CUtensorMap tm_q;    // fp16 Q   [T][hq][d], box {64, 1, 128}, 128B swizzle
   CUtensorMap tm_q8;   // int8 Q   [T][hq][d], box {d, 1, 128}
-  CUtensorMap tm_k;    // fp16 K   [T][hk][d], box {64, 1, 64}
+  CUtensorMap tm_k;    // fp16 K   [T][hk][d], box {64, 1, 64}, 128B swizzle
   CUtensorMap tm_k8;   // int8 K   [T][hk][d], box {d, 1, 64}
-  CUtensorMap tm_v;    // fp16 V   [T][hk][d], box {64, 1, 64}
+  CUtensorMap tm_v;    // fp16 V   [T][hk][d], box {64, 1, 64}, 128B swizzle
   void* o;
   float* lse;
   const int32_t* cu_seqlens;
@@ -136,8 +138,8 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        int* ticket, int fp8, cudaStream_t stream);
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
 int read_and_clear_status(unsigned int* status, cudaStream_t stream);
-// Device address of the allocation-free entry point's scratch array on the
-// current device (looked up once per device).
+// Device address of the allocation-free entry point's scratch array in the
+// calling thread's current context (looked up once per context).
 int noalloc_scratch(void** ptr);
 int launch_selftest_wait(unsigned long long timeout_ns, cudaStream_t stream);
 
