@@ -321,10 +321,11 @@ int tilemix_prefill_host(const tilemix_prefill_host_args* args, void* stream);
  * the quantisation pre-pass serve as the K cache, and a new token's query
  * reads the routing word of its query-tile row.  The pages give no decode
  * algorithm; this library reads it as the prefill method applied to one row:
- *   - sequence s holds seq_len[s] >= 1 cached tokens in cache rows
+ *   - sequence s holds seq_len[s] cached tokens in cache rows
  *     [seq_start[s], seq_start[s] + seq_len[s]); the new token is the last
  *     one, at position t = seq_len[s] - 1, its K and V already written, and it
- *     attends to positions 0..t (causal);
+ *     attends to positions 0..t (causal); a sequence with seq_len[s] = 0 has
+ *     no token and is skipped;
  *   - key tile kt (keys 64 kt .. 64 kt + 63) uses the INT8 score path iff bit
  *     (kt / g[s]) of masks[(qtile_start[s] + t / 128) * hk + kv] is set;
  *   - the query is quantised as a block of its own (one row: earlier queries
@@ -353,7 +354,9 @@ typedef struct tilemix_decode_args {
   float* k_scale;             /* device fp32 [hk][total_ktiles]: K block scales */
   void* o;                    /* device fp16 [nseq][hq][d] */
   const int32_t* seq_start;   /* device [nseq]: first cache row of each sequence */
-  const int32_t* seq_len;     /* device [nseq]: tokens in the cache incl. the new one, >= 1 */
+  const int32_t* seq_len;     /* device [nseq]: tokens in the cache incl. the new one; 0 = an
+                                 empty sequence: nothing is computed for it and its O rows
+                                 are left as they are */
   const int32_t* ktile_start; /* device [nseq]: k_scale column of each sequence's first K block */
   const int32_t* qtile_start; /* device [nseq]: masks row of each sequence's first query tile */
   const uint64_t* masks;      /* device [total_qtiles][hk] routing words */

@@ -15,6 +15,9 @@ MAX_ABS = 2e-3
 MEAN_ABS = 2e-4
 
 
+_INPUTS = {}
+
+
 class Case:
     def __init__(self, lengths, hq, hk, d, causal=True, template="band", percent=50, g=None,
                  outliers=0, lowrank=0, seed=0, routing_seed=0, kv_map=None):
@@ -47,8 +50,14 @@ class Case:
         return sum(self.lengths)
 
     def inputs(self):
-        return synth.make_qkv(self.seed, self.total_tokens, self.hq, self.hk, self.d,
-                              outliers=self.outliers, lowrank=self.lowrank)
+        # one draw per process and shape: the workload sweeps reuse it
+        key = (self.seed, self.total_tokens, self.hq, self.hk, self.d, self.outliers,
+               self.lowrank)
+        if key not in _INPUTS:
+            if len(_INPUTS) >= 2:
+                _INPUTS.clear()
+            _INPUTS[key] = synth.make_qkv(*key[:5], outliers=self.outliers, lowrank=self.lowrank)
+        return _INPUTS[key]
 
     def masks(self, words=None):
         if words is not None:

@@ -47,6 +47,8 @@ def _run(lengths, hq, hk, d, masks_fn, g, seed, slack=37, kv_map=None, tiles_per
         want_ks[:, ktiles[s]:ktiles[s] + sc.shape[1]] = sc
         k8[starts[s]:starts[s] + L] = c
         ks[:, ktiles[s]:ktiles[s] + sc.shape[1]] = sc
+        if L == 0:
+            continue
         b = (L - 1) // 64
         k8[starts[s] + 64 * b:starts[s] + L] = 99
         ks[:, ktiles[s] + b] = -1.0
@@ -55,15 +57,23 @@ def _run(lengths, hq, hk, d, masks_fn, g, seed, slack=37, kv_map=None, tiles_per
     dec = tm.TileMixDecode(starts, lengths, ktiles, qt[:-1], hq, hk, d, masks, g, total_kt,
                            kv_head_of_q=kv_map, device=dev, tiles_per_split=tiles_per_split)
     qd, kd, vd, k8d, ksd = t(q), t(k), t(v), t(k8), t(ks)
-    o = dec(qd, kd, vd, k8d, ksd)
+    o = dec(qd, kd, vd, k8d, ksd, o=torch.full_like(qd, float("nan")))
     torch.cuda.synchronize()
     assert tm.tilemix_get_error() == tm.OK
     got_k8, got_ks = k8d.cpu().numpy(), ksd.cpu().numpy()
     for s, L in enumerate(lengths):
         assert np.array_equal(got_k8[starts[s]:starts[s] + L], want_k8[starts[s]:starts[s] + L])
     assert np.array_equal(got_ks.view(np.uint32), want_ks.view(np.uint32))
-    want, _ = oracle.decode_rows(q, k, v, starts, lengths, masks, qt[:-1], g, kv_map=kv_map)
+    # an empty sequence has no token: nothing is computed for it and its O
+    # rows keep what they held
+    live = [s for s, L in enumerate(lengths) if L > 0]
     got = o.cpu().numpy().astype(np.float64)
+    for s, L in enumerate(lengths):
+        if L == 0:
+            assert np.isnan(got[s]).all()
+    want, _ = oracle.decode_rows(q[live], k, v, [starts[s] for s in live], [lengths[s] for s in live],
+                                 masks, qt[:-1][live], g[live], kv_map=kv_map)
+    got = got[live]
     assert np.isfinite(got).all()
     mx, mn = gc.errors(got.reshape(-1, d), want.reshape(-1, d))
     assert mx <= gc.MAX_ABS and mn <= gc.MEAN_ABS, (mx, mn)
@@ -119,6 +129,12 @@ def test_decode_group_sizes(group, d):
     lengths = [70, 257, 1]
     g = np.ones(len(lengths), dtype=np.int32)
     _run(lengths, 2 * group, 2, d, _template("sptrans", 75, lengths, 2, g), g, seed=10 + group)
+
+
+def test_decode_zero_length_sequences():
+    lengths = [0, 70, 0, 200, 0]
+    g = np.ones(len(lengths), dtype=np.int32)
+    _run(lengths, 4, 2, 128, _template("sptrans", 75, lengths, 2, g), g, seed=11)
 
 
 @pytest.mark.parametrize("tps", [1, 3, 5, 16, 64])

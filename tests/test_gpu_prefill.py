@@ -233,16 +233,16 @@ def test_gqa_head_map():
 
 # -------------------------------------------- full workloads, sampled rows ---
 
+# The coverage x layout sweep: every template at 25, 50 and 75% INT8.
+SWEEP = [("sweep_8k_b8", dict(template=t, percent=pct))
+         for t in ("band", "global", "row_random", "aligned_sparse", "bigbird", "sptrans")
+         for pct in (25, 50, 75)]
+
 WORKLOAD_RUNS = [
     ("llama3b_4k_b8", dict()),
     ("llama3b_4k_b8", dict(percent=0)),
     ("llama3b_4k_b8", dict(percent=100)),
-    ("sweep_8k_b8", dict(template="band", percent=25)),
-    ("sweep_8k_b8", dict(template="global", percent=75)),
-    ("sweep_8k_b8", dict(template="row_random", percent=50)),
-    ("sweep_8k_b8", dict(template="aligned_sparse", percent=25)),
-    ("sweep_8k_b8", dict(template="bigbird", percent=75)),
-    ("sweep_8k_b8", dict(template="sptrans", percent=50)),
+] + SWEEP + [
     ("varlen_qwen7b", dict()),
     ("long_64k", dict()),
 ]
@@ -267,6 +267,59 @@ def test_workload_sampled_rows(name, over):
         rows = gc.sample_rows(case.lengths, case.hq, per_head_random=32)
     want, _, _ = gc.oracle_rows(case, q, k, v, masks, rows)
     _check_out(case, out["o"], want, rows)
+
+
+# ------------------------------------------------------ packed batches ---
+
+def test_zero_length_sequences_in_a_batch():
+    # Empty sequences hold no tiles, rows or words; the device's sequence
+    # lookups skip them.  Full parity on every row, and the host-buffer call
+    # (runs of whole sequences, some of them empty) equals the device call.
+    import tile_routed_mixed_b200 as tm
+    case = gc.Case([0, 300, 0, 0, 129, 0], 4, 2, 128, template="sptrans", percent=75, seed=12)
+    q, k, v = case.inputs()
+    masks = case.masks()
+    out = gc.run_gpu(case, q, k, v, masks, lse=True)
+    rows = oracle.all_rows(case.lengths, case.hq)
+    want, lse, _ = gc.oracle_rows(case, q, k, v, masks, rows)
+    _check_out(case, out["o"], want, rows)
+    cu = np.concatenate([[0], np.cumsum(case.lengths)])
+    assert np.abs(out["lse"][rows[:, 1], cu[rows[:, 0]] + rows[:, 2]] - lse).max() < 2e-3
+    pf = tm.TileMixPrefill(case.lengths, case.hq, case.hk, case.d, masks, case.g)
+    qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    for chunks in (1, 3, 6):
+        oh = torch.full(q.shape, float("nan"), dtype=torch.float16).pin_memory()
+        qd, kd, vd = (torch.empty(x.shape, dtype=torch.float16, device="cuda") for x in (q, k, v))
+        od = torch.empty(q.shape, dtype=torch.float16, device="cuda")
+        pf.from_host(qh, kh, vh, oh, qd, kd, vd, od, chunks=chunks)
+        torch.cuda.current_stream().synchronize()
+        assert tm.tilemix_get_error() == tm.OK
+        assert np.array_equal(oh.numpy().view(np.uint16), out["o"].view(np.uint16))
+
+
+def test_head_map_entry_out_of_range_is_reported_and_skipped():
+    # Query head 2 names KV head 2 of 2: its work items are skipped (its O
+    # rows stay as they were) and the status word reports INVALID_ARG; the
+    # other heads are computed as usual.
+    import tile_routed_mixed_b200 as tm
+    kv_map = np.array([0, 1, 2, 1], dtype=np.int32)
+    good_map = np.array([0, 1, 0, 1], dtype=np.int32)
+    case = gc.Case([300, 200], 4, 2, 128, kv_map=good_map, seed=13)
+    q, k, v = case.inputs()
+    masks = case.masks()
+    pf = tm.TileMixPrefill(case.lengths, case.hq, case.hk, case.d, masks, case.g,
+                           kv_head_of_q=kv_map)
+    qd, kd, vd = (torch.from_numpy(x).cuda() for x in (q, k, v))
+    od = torch.full_like(qd, float("nan"))
+    pf(qd, kd, vd, od)
+    assert tm.tilemix_get_error() == tm.ERR_INVALID_ARG
+    assert tm.tilemix_get_error() == tm.OK
+    got = od.cpu().numpy()
+    assert np.isnan(got[:, 2]).all()
+    rows = oracle.all_rows(case.lengths, case.hq)
+    rows = rows[rows[:, 1] != 2]
+    want, _, _ = gc.oracle_rows(case, q, k, v, masks, rows)
+    _check_out(case, got, want, rows)
 
 
 # ------------------------------------------------------------- failures ---

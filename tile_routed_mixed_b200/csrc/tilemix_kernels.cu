@@ -38,31 +38,26 @@ constexpr int BN = 64;   // keys per tile
 // Persistent CTAs, one per SM, each walking a share of the work items: one
 // item per (sequence, query head, pair of query-tile rows 2j and 2j+1),
 // heaviest pairs first.  The two 128-row Q tiles of an item share every K/V
-// tile load.  Per Q tile, key tile t's scores S(t) go to one of two TMEM
-// score buffers (t alternating), the softmax turns them into P (fp16) over the
-// same columns, and P.V accumulates into O.  The MMA thread of a Q tile issues
-// P(t).V and then S(t + 2) = Q K(t + 2)^T into the buffer P(t) just left, so
-// S(t + 1) is ready while the softmax works on tile t and S(t + 2) is computed
-// while it works on tile t + 1: the softmax never waits for the tensor cores
-// as long as one tile's P.V and QK^T take less time than one tile's softmax.
+// tile load; the K/V ring, the score and P buffers run on across items, so
+// one item's last tiles and epilogue overlap the next item's first tiles.
 // Warp roles (12 warps, three warpgroups):
-//   warp 0      TMA producer: both Q tiles (fp16 and int8), then the item's
-//               ring entries: entry e holds key tile e in each precision the
-//               two rows' routing bits need and the fp16 V of key tile e - 2,
-//               the operands of one MMA step [P(e - 2).V, S(e)]
+//   warp 0      TMA producer: both Q tiles (fp16 and int8), then per key tile
+//               the K tile in each precision the two rows' routing bits need,
+//               and the fp16 V tile
 //   warps 1, 2  MMA issuers of Q tile 0 and Q tile 1 (warp 1 also owns TMEM):
-//               per entry, O_q += P_q(e - 2) V (kind::f16, P read from TMEM),
-//               then S_q(e) = Q_q K(e)^T (kind::f16 -> f32 or kind::i8 -> s32,
-//               by row q's routing bit)
+//               S_q = Q_q K^T (kind::f16 -> f32 or kind::i8 -> s32, by row
+//               q's routing bit) into one of the two TMEM score buffers of Q
+//               tile q, then O_q += P_q V (kind::f16, P read from TMEM)
 //   warps 4-7   softmax of Q tile 0, warps 8-11 softmax of Q tile 1: one query
 //               row per thread; routed scores -> float score domain, legality
 //               mask, online max / normaliser, P in fp16 back to TMEM; when a
 //               row's running max moved (rare with lazy rescaling), the warp
-//               rescales its rows of O in TMEM first; at the end O / l in fp16
-// TMEM (512 columns): per Q tile q, O_q [D cols] at column 256 q and its two
-// 64-column score buffers at 256 q + 128 and 256 q + 192 (P in the first 32
-// columns of the buffer its S came from).
+//               rescales its rows of O in TMEM after the previous P.V landed,
+//               before P is handed to the next P.V; at the end O / l in fp16
+// TMEM (512 columns): per Q tile q, O_q [D cols] and two 64-column score
+// buffers, at column offset 256 q.
 // ===================================================================
+constexpr int kStages = 3;
 constexpr int kPrefillThreads = 384;
 // No register split: every role fits in the registers the launch gives
 // each of the 384 threads.
@@ -73,7 +68,6 @@ constexpr int kSoftmaxWarp0 = 4;
 // stale max only shifts fp16 underflow further below the true maximum.
 constexpr float kRescaleThreshold = 15.0f;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxEntries = 6;
 
 template <int D>
 struct Smem {
@@ -82,54 +76,49 @@ struct Smem {
   static constexpr int kK16 = BN * D * 2;     // fp16 K tile
   static constexpr int kK8 = BN * D;          // int8 K tile
   static constexpr int kV = BN * D * 2;       // fp16 V tile
-  static constexpr int kEntry = kK16 + kK8 + kV;
-  static constexpr int kEntries = D == 128 ? 3 : 6;
   static constexpr int kOffQ = 0;                          // + q * kQ
   static constexpr int kOffQ8 = kOffQ + 2 * kQ;            // + q * kQ8
-  static constexpr int kOffRing = kOffQ8 + 2 * kQ8;        // + entry * kEntry
-  static constexpr int kOffBar = kOffRing + kEntries * kEntry;
+  static constexpr int kOffK16 = kOffQ8 + 2 * kQ8;         // + stage * kK16
+  static constexpr int kOffK8 = kOffK16 + kStages * kK16;  // + stage * kK8
+  static constexpr int kOffV = kOffK8 + kStages * kK8;     // + stage * kV
+  static constexpr int kOffBar = kOffV + kStages * kV;
   static constexpr int kBytes = kOffBar + 512 + 1024;      // + alignment slack
-  // inside an entry
-  static constexpr int kEK16 = 0, kEK8 = kK16, kEV = kK16 + kK8;
+  static constexpr int kF16Steps = D / 16;
+  static constexpr int kI8Steps = D / 32;
   static constexpr uint32_t kI8Layout = D == 128 ? ptx::kSwizzle128B : ptx::kSwizzle64B;
   static constexpr uint32_t kI8Sbo = 8 * D;  // 8 rows of D bytes
+  // TMEM columns of Q tile q: O [D], S [64], P buffers 0 and 1 [32 each]
   __host__ __device__ static constexpr uint32_t col_o(int q) { return 256u * q; }
-  __host__ __device__ static constexpr uint32_t col_b(int q, int b) {
-    return 256u * q + 128u + 64u * b;
+  __host__ __device__ static constexpr uint32_t col_s(int q) { return 256u * q + D; }
+  __host__ __device__ static constexpr uint32_t col_p(int q, int b) {
+    return 256u * q + D + 64u + 32u * b;
   }
 };
-static_assert(Smem<128>::kBytes <= 232448 && Smem<64>::kBytes <= 232448,
-              "shared memory exceeds the 227 KB a CTA may use");
-static_assert(Smem<64>::kEntries <= kMaxEntries && Smem<128>::kEntries <= kMaxEntries,
-              "entry barriers");
 
 // Every mbarrier below is waited on by parity.  A parity wait is only
 // unambiguous when the waiter is at most one phase behind the barrier; for
 // each wait, the barrier's next phase needs an event that cannot happen before
 // the waiter has moved on (noted at the waits).  The CTA is persistent, so the
-// phases run on across work items: each role keeps running counts.  S and P
-// have one barrier per score buffer: S(t) and S(t + 1) are both issued before
-// the softmax reads either, so one barrier for both could run two phases
-// ahead of its waiter.
-//   S(t + 2) goes into the buffer of P(t).  The MMA thread issues it right
-//   after P(t).V, which waited for p_full(t) (the softmax has read S(t) and
-//   written P(t) by then), and the tensor pipe runs one thread's MMAs in
-//   order, so P(t).V reads P(t) before S(t + 2) overwrites it.  The commit
-//   that signals S(t + 1) covers P(t - 1).V (issued before it).
+// phases run on across work items: each role keeps running counts.
+//   S is single-buffered: S(n+1) needs s_free(n), i.e. the softmax has read
+//   S(n).  P is double-buffered; the softmax stores P(n) only after S(n)
+//   landed, and the MMA thread issues S(n) after P(n-2).V, so that commit
+//   covers P(n-2).V: the MMA thread cannot fall two phases behind p_full.
 struct Barriers {
-  uint64_t q_full[2];                // Q tile q (fp16 and int8) of the current item landed
-  uint64_t q_free[2];                // the last S = Q K^T of Q tile q's item completed
-  uint64_t e_full[kMaxEntries];      // a ring entry's tiles landed
-  uint64_t e_empty[kMaxEntries];     // both MMA threads are done with a ring entry
-  uint64_t s_full[2][2];             // S_q in TMEM score buffer b (one phase per use)
-  uint64_t p_full[2][2];             // P_q in buffer b (and O_q rescaled if needed)
-  uint64_t pv_last[2];               // P.V of the item's second-to-last tile completed
-  uint64_t o_final[2];               // the last P.V of Q tile q's item completed
-  uint64_t o_free[2];                // the softmax has read O_q of the item out of TMEM
+  uint64_t q_full[2];          // Q tile q (fp16 and int8) of the current item landed
+  uint64_t q_free[2];          // the last S = Q K^T of Q tile q's item completed
+  uint64_t kv_full[kStages];   // K (each precision needed) and V of a key tile landed
+  uint64_t kv_empty[kStages];  // both MMA threads are done with that key tile
+  uint64_t s_full[2];          // S_q in TMEM
+  uint64_t s_free[2];          // S_q read out: the S columns may be refilled
+  uint64_t p_full[2][2];       // P_q in TMEM buffer b (and O_q rescaled if needed)
+  uint64_t pv_done[2][2];      // the P.V reading P_q buffer b completed
+  uint64_t o_final[2];         // the last P.V of Q tile q's item completed
+  uint64_t o_free[2];          // the softmax has read O_q of the item out of TMEM
   uint64_t drain[2];
-  uint64_t item_full[4];             // a work item index published in ring slot k % 4
-  uint64_t item_empty[4];            // every consumer has read ring slot k % 4
-  int item_ring[4];                  // item indices, -1 = no more work
+  uint64_t item_full[4];       // a work item index published in ring slot k % 4
+  uint64_t item_empty[4];      // every consumer has read ring slot k % 4
+  int item_ring[4];            // item indices, -1 = no more work
   uint32_t tmem_base;
   int abort;
 };
@@ -169,6 +158,7 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// Drain wait used on the way out: ignores the abort flag, still bounded.
 // A consumer's next work item from ring slot k % 4 (item_full's next phase
 // for the slot needs this consumer's item_empty arrival): the index, -1 when
 // there is no more work, or kItemAbort if the wait gave up.
@@ -185,7 +175,6 @@ __device__ __forceinline__ int next_item(Barriers* bars, uint32_t k, volatile in
   return w;
 }
 
-// Drain wait used on the way out: ignores the abort flag, still bounded.
 __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity,
                                           unsigned long long timeout_ns) {
   const unsigned long long start = ptx::globaltimer();
@@ -368,41 +357,41 @@ struct SoftmaxCtx {
   Barriers* bars;
   volatile int* abort_flag;
   unsigned long long tmo;
-  uint32_t tb, to;  // TMEM addresses of this lane's score buffer 0 and O
+  uint32_t ts, to, tp0;           // TMEM addresses of this lane's S, O and P buffer 0
   int q, L, row0, my_row, h, t0, ntq;
   float q_sc;
-  const float* ks;  // K block scales of the sequence and KV head
+  const float* ks;                // K block scales of the sequence and KV head
 };
 struct RowState {
   float m;          // running max, log2 units
   float l;          // normaliser: sum of the fp16-rounded P actually used in P.V
   float k_sc_next;  // K scale of the next key tile (loaded one tile ahead)
-  uint32_t n_s;     // S_q read so far (tile t's buffer is n_s & 1)
-  uint32_t n_pvl;   // pv_last phases before this item
+  uint32_t n_s;     // S_q read so far
+  uint32_t n_p;     // P_q stored so far
 };
 
 // One key tile of the shared online softmax for this thread's row: S from
 // TMEM, the routed score domain, legality, max / normaliser update, lazy
-// rescale of O, P (fp16) over the first columns of S's buffer.  kMask adds the
-// legality mask that only the diagonal and sequence-tail tiles need, kDebug
-// the INT32 score dump of debug runs; the lean copy runs every other tile, so
-// the hot loop carries no code for them.  False if a wait gave up.
+// rescale of O, P (fp16) to TMEM.  kMask adds the legality mask that only the
+// diagonal and sequence-tail tiles need, kDebug the INT32 score dump of debug
+// runs; the lean copy runs every other tile, so the hot loop carries no code
+// for them.  False if a wait gave up.
 template <int D, bool kMask, bool kDebug, bool kFp8>
 __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st, int i, bool is_int,
                                              uint32_t (&r)[64]) {
   const int q = cx.q;
+  const int sb = st.n_p & 1;
   const float k_sc = st.k_sc_next;
   if (i + 1 < cx.ntq) st.k_sc_next = __ldg(cx.ks + i + 1);
-  // this buffer's s_full next phase needs S(i + 2), issued after P(i).V,
-  // which needs p_full from this tile
-  const int buf = st.n_s & 1;
-  if (!wait_bar_warp(&cx.bars->s_full[q][buf], (st.n_s >> 1) & 1, cx.abort_flag, cx.tmo))
-    return false;
+  // s_full's next phase needs s_free from this read
+  if (!wait_bar_warp(&cx.bars->s_full[q], st.n_s & 1, cx.abort_flag, cx.tmo)) return false;
   ptx::tc_fence_after();
-  const uint32_t tb = cx.tb + 64u * buf;
-  ptx::tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  ptx::tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  ptx::tmem_ld32(cx.ts, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  ptx::tmem_ld32(cx.ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
   ptx::tmem_ld_wait();
+  // S is in registers: the MMA warp may compute the next S now
+  ptx::tc_fence_before();
+  ptx::mbar_arrive(&cx.bars->s_free[q]);
   ++st.n_s;
   const int key0 = i * BN;
   if (kDebug && !kFp8 && is_int && cx.p->dbg && cx.my_row < cx.L) {
@@ -466,17 +455,13 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st,
   st.l = st.l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
   st.m = m_use;
   if (i > 0 && __any_sync(0xffffffffu, resc)) {
-    // O holds P.V of tiles < i: rescale this warp's rows (rows without a max
-    // move multiply by 1) once P(i - 1).V completed.  The commit that signals
-    // S(i + 1) covers it (S(i + 1) was issued after P(i - 1).V); the item's
-    // last tile has no S(i + 1) and waits for pv_last instead.  Neither
-    // barrier can move past the awaited phase before p_full of this tile.
-    const bool ok =
-        i + 1 < cx.ntq
-            ? wait_bar_warp(&cx.bars->s_full[q][st.n_s & 1], (st.n_s >> 1) & 1, cx.abort_flag,
-                            cx.tmo)
-            : wait_bar_warp(&cx.bars->pv_last[q], st.n_pvl & 1, cx.abort_flag, cx.tmo);
-    if (!ok) return false;
+    // O holds P.V of tiles < i: rescale this warp's rows once P(i-1).V has
+    // landed (rows without a max move multiply by 1).  The P.V of the previous
+    // tile is the (n_p - 1)-th; the next phase of its pv_done barrier needs
+    // p_full from this tile.
+    if (!wait_bar_warp(&cx.bars->pv_done[q][(st.n_p - 1) & 1], ((st.n_p - 1) >> 1) & 1,
+                       cx.abort_flag, cx.tmo))
+      return false;
     ptx::tc_fence_after();
 #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -488,11 +473,14 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& cx, RowState& st,
       ptx::tmem_st32(cx.to + cc * 32, o);
     }
   }
-  // P over the first 32 columns of S's buffer (already read out)
-  ptx::tmem_st32(tb, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
+  // P buffer sb held the P stored two tiles ago.  Its P.V was issued before
+  // this tile's S by the same thread, and the commit that signalled S covers
+  // every MMA issued before it: no wait needed.
+  ptx::tmem_st32(cx.tp0 + 32 * sb, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
   ptx::tmem_st_wait();
   ptx::tc_fence_before();
-  ptx::mbar_arrive(&cx.bars->p_full[q][buf]);
+  ptx::mbar_arrive(&cx.bars->p_full[q][sb]);
+  ++st.n_p;
   return true;
 }
 
@@ -515,20 +503,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int num_items = p.max_qpairs * p.nseq * p.hq;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S::kEntries; ++i) {
-      ptx::mbar_init(&bars->e_full[i], 1);
-      ptx::mbar_init(&bars->e_empty[i], 2);  // one commit per MMA thread and use
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&bars->kv_full[i], 1);
+      ptx::mbar_init(&bars->kv_empty[i], 2);  // one commit per MMA thread and key tile
     }
     for (int q = 0; q < 2; ++q) {
       ptx::mbar_init(&bars->q_full[q], 1);
       ptx::mbar_init(&bars->q_free[q], 1);
-      for (int b = 0; b < 2; ++b) {
-        ptx::mbar_init(&bars->s_full[q][b], 1);
-        ptx::mbar_init(&bars->p_full[q][b], 128);
+      for (int i = 0; i < 2; ++i) {
+        ptx::mbar_init(&bars->p_full[q][i], 128);
+        ptx::mbar_init(&bars->pv_done[q][i], 1);
       }
-      ptx::mbar_init(&bars->pv_last[q], 1);
       ptx::mbar_init(&bars->o_final[q], 1);
       ptx::mbar_init(&bars->o_free[q], 128);
+      ptx::mbar_init(&bars->s_full[q], 1);
+      ptx::mbar_init(&bars->s_free[q], 128);
       ptx::mbar_init(&bars->drain[q], 1);
     }
     for (int i = 0; i < kItemSlots; ++i) {
@@ -551,38 +540,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   if (warp == 0) {
     // ================= TMA producer =================
-    // Per item: each Q tile (fp16 and int8) once its slot is free, then ring
-    // entries e = 0 .. nt + 1: key tile e in each precision the two rows'
-    // routing bits need (e < nt) and the fp16 V of key tile e - 2 (e >= 2).
-    // The ring runs on across items.
+    // Per item: each Q tile (fp16 and int8) once its slot is free, then per
+    // key tile the K tile in each precision the two rows' routing bits need
+    // and the fp16 V tile, into the 3-stage ring, which runs on across items.
     if (lane == 0) {
       ptx::prefetch_tensormap(&p.tm_q);
       ptx::prefetch_tensormap(&p.tm_q8);
       ptx::prefetch_tensormap(&p.tm_k);
       ptx::prefetch_tensormap(&p.tm_k8);
       ptx::prefetch_tensormap(&p.tm_v);
-      uint32_t pos = 0;                   // ring entries filled so far
+      uint32_t kv_tiles = 0;              // key tiles issued so far (ring position)
       uint32_t q_loads[2] = {0u, 0u};     // loads of each Q slot so far
       bool ok = true;
-      for (uint32_t n = 0; ok; ++n) {
-        int w = n == 0 ? static_cast<int>(blockIdx.x)
+      for (uint32_t k = 0; ok; ++k) {
+        int w = k == 0 ? static_cast<int>(blockIdx.x)
                        : static_cast<int>(gridDim.x) + atomicAdd(p.ticket, 1);
         if (w >= num_items) w = -1;
         // publish it once every consumer has read the slot's previous item
         // (item_empty's next phase needs this publication)
-        const int islot = n % kItemSlots;
-        if (n >= kItemSlots &&
-            !wait_bar(&bars->item_empty[islot], ((n / kItemSlots) - 1) & 1, abort_flag, tmo))
+        const int slot = k % kItemSlots;
+        if (k >= kItemSlots &&
+            !wait_bar(&bars->item_empty[slot], ((k / kItemSlots) - 1) & 1, abort_flag, tmo))
           break;
-        *reinterpret_cast<volatile int*>(&bars->item_ring[islot]) = w;
-        ptx::mbar_arrive(&bars->item_full[islot]);
+        *reinterpret_cast<volatile int*>(&bars->item_ring[slot]) = w;
+        ptx::mbar_arrive(&bars->item_full[slot]);
         if (w < 0) break;
         WorkItem it;
         if (!load_item(p, w, it)) continue;
         // Q tile q's slot is refilled once the previous item's last S of it
         // completed (q_free's next phase needs this load).  Q tile 1 goes
-        // after the item's first entry, so that Q tile 0 can start the item
-        // while Q tile 1 still finishes the previous one.
+        // after the item's first key tile, so that the shorter Q tile 0 can
+        // start the item while Q tile 1 still finishes the previous one.
         const auto load_q = [&](int q) {
           if (q_loads[q] > 0 &&
               !wait_bar(&bars->q_free[q], (q_loads[q] - 1) & 1, abort_flag, tmo))
@@ -599,57 +587,51 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         };
         if (!load_q(0)) break;
         GroupCursor gc;
-        for (int e = 0; ok && e < it.nt + 2; ++e) {
-          const int sl = pos % S::kEntries;
-          // the entry's previous use released by both MMA threads
-          // (e_empty's next phase needs this entry's next load)
-          if (pos >= static_cast<uint32_t>(S::kEntries) &&
-              !wait_bar(&bars->e_empty[sl], ((pos / S::kEntries) - 1) & 1, abort_flag, tmo)) {
+        for (int i = 0; ok && i < it.nt; ++i, gc.next(it.gs)) {
+          const int st = kv_tiles % kStages;
+          // K precisions the two rows need for this tile (at least one: i < nt)
+          const bool b0 = gc.int8(it.w0), b1 = gc.int8(it.w1);
+          const bool need8 = (i < it.nt0 && b0) || (i < it.nt1 && b1);
+          const bool need16 = (i < it.nt0 && !b0) || (i < it.nt1 && !b1);
+          // the stage's previous tile released by both MMA threads
+          if (kv_tiles >= kStages &&
+              !wait_bar(&bars->kv_empty[st], ((kv_tiles / kStages) - 1) & 1, abort_flag, tmo)) {
             ok = false;
             break;
           }
-          bool need16 = false, need8 = false;
-          if (e < it.nt) {
-            // K precisions the two rows need for key tile e (at least one)
-            const bool b0 = gc.int8(it.w0), b1 = gc.int8(it.w1);
-            need8 = (e < it.nt0 && b0) || (e < it.nt1 && b1);
-            need16 = (e < it.nt0 && !b0) || (e < it.nt1 && !b1);
-            gc.next(it.gs);
-          }
-          const bool needv = e >= 2;
-          uint64_t* full = &bars->e_full[sl];
-          uint8_t* ent = smem + S::kOffRing + sl * S::kEntry;
-          ptx::mbar_expect_tx(full, (need16 ? S::kK16 : 0) + (need8 ? S::kK8 : 0) +
-                                        (needv ? S::kV : 0));
-          const int keyk = it.t0 + e * BN, keyv = it.t0 + (e - 2) * BN;
+          const int key0 = it.t0 + i * BN;
+          uint64_t* full = &bars->kv_full[st];
+          ptx::mbar_expect_tx(full, (need16 ? S::kK16 : 0) + (need8 ? S::kK8 : 0) + S::kV);
           if (need16) {
 #pragma unroll
             for (int j = 0; j < D / 64; ++j)
-              ptx::tma_load_3d(ent + S::kEK16 + j * BN * 128, &p.tm_k, full, j * 64, it.kv, keyk);
+              ptx::tma_load_3d(smem + S::kOffK16 + st * S::kK16 + j * BN * 128, &p.tm_k, full,
+                               j * 64, it.kv, key0);
           }
-          if (need8) ptx::tma_load_3d(ent + S::kEK8, &p.tm_k8, full, 0, it.kv, keyk);
-          if (needv) {
+          if (need8)
+            ptx::tma_load_3d(smem + S::kOffK8 + st * S::kK8, &p.tm_k8, full, 0, it.kv, key0);
 #pragma unroll
-            for (int j = 0; j < D / 64; ++j)
-              ptx::tma_load_3d(ent + S::kEV + j * BN * 128, &p.tm_v, full, j * 64, it.kv, keyv);
-          }
-          ++pos;
-          if (e == 0 && it.nq == 2 && !load_q(1)) ok = false;
+          for (int j = 0; j < D / 64; ++j)
+            ptx::tma_load_3d(smem + S::kOffV + st * S::kV + j * BN * 128, &p.tm_v, full, j * 64,
+                             it.kv, key0);
+          ++kv_tiles;
+          if (i == 0 && it.nq == 2 && !load_q(1)) ok = false;
         }
       }
       // Never leave with copies into this CTA's shared memory in flight.
       for (int q = 0; q < 2; ++q)
         if (q_loads[q] > 0) drain_bar(&bars->q_full[q], (q_loads[q] - 1) & 1, tmo);
-      for (uint32_t sl = 0; sl < static_cast<uint32_t>(S::kEntries) && sl < pos; ++sl)
-        drain_bar(&bars->e_full[sl], ((pos - 1 - sl) / S::kEntries) & 1, tmo);
+      for (uint32_t st = 0; st < kStages && st < kv_tiles; ++st)
+        drain_bar(&bars->kv_full[st], ((kv_tiles - 1 - st) / kStages) & 1, tmo);
     }
   } else if (warp == 1 || warp == 2) {
     // ================= MMA issuers: warp 1 for Q tile 0, warp 2 for Q tile 1 =====
-    // Per item and ring entry e: P_q(e - 2).V once the softmax posted it, then
-    // S_q(e) into the score buffer P_q(e - 2) occupied.  Each thread releases
-    // every entry of every item (count 2 per entry) with one commit after its
-    // MMAs, or once the entry has landed if its Q tile does not use it (so
-    // that the arrival cannot count towards the entry's previous use).
+    // Per item, in key-tile order: S_q(0), then per key tile j: S_q(j + 1) as
+    // soon as the softmax has read S_q(j) out of TMEM, then P_q(j).V once the
+    // softmax has posted P_q(j).  Each thread releases every key tile of every
+    // item (count 2 per stage): after its P.V, or once the tile has landed if
+    // its Q tile does not use it (so that the arrival cannot count towards
+    // the stage's previous tile).
     const int q = warp - 1;
     if (lane == 0) {
       const uint32_t a_smem = ptx::smem_addr(smem);
@@ -659,14 +641,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint32_t aq16 = a_smem + S::kOffQ + q * S::kQ;
       const uint32_t aq8 = a_smem + S::kOffQ8 + q * S::kQ8;
       const uint32_t d_o = tmem + S::col_o(q);
-      const uint32_t d_b = tmem + S::col_b(q, 0);
-      uint32_t pos = 0;       // ring entries consumed so far
-      uint32_t n_s = 0;       // S_q issued so far (the next one's buffer is n_s & 1)
+      const uint32_t d_s = tmem + S::col_s(q);
+      uint32_t kv_tiles = 0;  // key tiles of earlier items (ring position)
+      uint32_t n_s = 0;       // S_q issued so far
       uint32_t n_p = 0;       // P_q.V issued so far
       uint32_t n_items = 0;   // items that had a Q tile q
       bool ok = true;
-      for (uint32_t n = 0; ok; ++n) {
-        const int w = next_item(bars, n, abort_flag, tmo, false);
+      for (uint32_t k = 0; ok; ++k) {
+        const int w = next_item(bars, k, abort_flag, tmo, false);
         if (w == kItemAbort) {
           ok = false;
           break;
@@ -682,63 +664,72 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           ok = false;
           break;
         }
-        GroupCursor gc;  // routing group of key tile e
-        for (int e = 0; e < it.nt + 2; ++e, ++pos) {
-          const int sl = pos % S::kEntries;
-          if (!wait_bar(&bars->e_full[sl], (pos / S::kEntries) & 1, abort_flag, tmo)) {
-            ok = false;
-            break;
-          }
-          const uint32_t ent = a_smem + S::kOffRing + sl * S::kEntry;
-          const int jv = e - 2;  // V tile of the entry
-          if (jv >= 0 && jv < ntq) {
-            const int valid = it.L - jv * BN;
-            if (valid < BN) {
-              // Keys past the sequence end belong to the next packed
-              // sequence: zero their V rows so that 0 * (NaN or Inf) cannot
-              // reach O.  Both Q tiles write the same zeros, each before its
-              // own P.V.
-              uint8_t* vt = smem + S::kOffRing + sl * S::kEntry + S::kEV;
-              for (int part = 0; part < D / 64; ++part)
-                for (int r = valid; r < BN; ++r) {
-                  uint4* row = reinterpret_cast<uint4*>(vt + part * BN * 128 + r * 128);
-#pragma unroll
-                  for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
-                }
-              ptx::fence_proxy_async_smem();
-            }
-            // the first P.V of an item overwrites O_q: the previous item's
-            // epilogue must have read it (o_free's next phase needs this
-            // item's o_final)
-            if (jv == 0 && n_items > 0 &&
-                !wait_bar(&bars->o_free[q], (n_items - 1) & 1, abort_flag, tmo)) {
+        GroupCursor gc;  // routing group of tile i
+        for (int i = 0; i <= it.nt; ++i) {
+          if (i < it.nt) {
+            const uint32_t t = kv_tiles + i;
+            // S(n) overwrites S(n - 1) once the softmax has read it out
+            if (i < ntq && n_s > 0 && !wait_bar(&bars->s_free[q], (n_s - 1) & 1, abort_flag, tmo)) {
               ok = false;
               break;
             }
-            // this buffer's p_full next phase needs S(jv + 2), issued below
-            if (!wait_bar(&bars->p_full[q][n_p & 1], (n_p >> 1) & 1, abort_flag, tmo)) {
+            if (!wait_bar(&bars->kv_full[t % kStages], (t / kStages) & 1, abort_flag, tmo)) {
               ok = false;
               break;
             }
-            ptx::tc_fence_after();
-            issue_pv<D>(d_o, d_b + 64u * (n_p & 1), ent + S::kEV, tv, jv == 0);
-            ++n_p;
-            if (jv == ntq - 2) ptx::mma_commit(&bars->pv_last[q]);
-            if (jv == ntq - 1) ptx::mma_commit(&bars->o_final[q]);
-          }
-          if (e < it.nt) {
-            if (e < ntq) {
+            if (i < ntq) {
               ptx::tc_fence_after();
-              issue_qk<D, kFp8>(d_b + 64u * (n_s & 1), gc.int8(word), aq16, aq8, ent + S::kEK16,
-                                ent + S::kEK8, t16, t8);
-              ptx::mma_commit(&bars->s_full[q][n_s & 1]);
+              const int st = t % kStages;
+              issue_qk<D, kFp8>(d_s, gc.int8(word), aq16, aq8, a_smem + S::kOffK16 + st * S::kK16,
+                          a_smem + S::kOffK8 + st * S::kK8, t16, t8);
+              ptx::mma_commit(&bars->s_full[q]);
               ++n_s;
-              if (e == ntq - 1) ptx::mma_commit(&bars->q_free[q]);
+              if (i == ntq - 1) ptx::mma_commit(&bars->q_free[q]);
             }
             gc.next(it.gs);
           }
-          ptx::mma_commit(&bars->e_empty[sl]);
+          if (i >= 1) {
+            const int j = i - 1;
+            const int st = (kv_tiles + j) % kStages;
+            if (j < ntq) {
+              const int valid = it.L - j * BN;
+              if (valid < BN) {
+                // Keys past the sequence end belong to the next packed
+                // sequence: zero their V rows so that 0 * (NaN or Inf) cannot
+                // reach O.  Both Q tiles write the same zeros, each before its
+                // own P.V.
+                uint8_t* vslot = smem + S::kOffV + st * S::kV;
+                for (int part = 0; part < D / 64; ++part)
+                  for (int r = valid; r < BN; ++r) {
+                    uint4* row = reinterpret_cast<uint4*>(vslot + part * BN * 128 + r * 128);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+                  }
+                ptx::fence_proxy_async_smem();
+              }
+              // the first P.V of an item overwrites O_q: the previous item's
+              // epilogue must have read it (o_free's next phase needs this
+              // item's o_final)
+              if (j == 0 && n_items > 0 &&
+                  !wait_bar(&bars->o_free[q], (n_items - 1) & 1, abort_flag, tmo)) {
+                ok = false;
+                break;
+              }
+              const int pb = n_p & 1;
+              if (!wait_bar(&bars->p_full[q][pb], (n_p >> 1) & 1, abort_flag, tmo)) {
+                ok = false;
+                break;
+              }
+              ptx::tc_fence_after();
+              issue_pv<D>(d_o, tmem + S::col_p(q, pb), a_smem + S::kOffV + st * S::kV, tv, j == 0);
+              ptx::mma_commit(&bars->pv_done[q][pb]);
+              ++n_p;
+              if (j == ntq - 1) ptx::mma_commit(&bars->o_final[q]);
+            }
+            ptx::mma_commit(&bars->kv_empty[st]);
+          }
         }
+        kv_tiles += it.nt;
         if (mine) ++n_items;
       }
       // all MMAs of this thread complete before TMEM and shared memory go away
@@ -751,12 +742,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int tr = threadIdx.x - (kSoftmaxWarp0 + 4 * q) * 32;  // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     uint32_t n_s = 0;      // S_q read so far
-    uint32_t n_pvl = 0;    // pv_last phases so far
+    uint32_t n_p = 0;      // P_q stored so far
     uint32_t n_items = 0;  // items that had a Q tile q
     bool ok = true;
     uint32_t r[64];
-    for (uint32_t n = 0; ok; ++n) {
-      const int w = next_item(bars, n, abort_flag, tmo, true);
+    for (uint32_t k = 0; ok; ++k) {
+      const int w = next_item(bars, k, abort_flag, tmo, true);
       if (w == kItemAbort) {
         ok = false;
         break;
@@ -765,20 +756,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       WorkItem it;
       if (!load_item(p, w, it)) continue;
       if (q >= it.nq) continue;
-      const int h = it.h, kv = it.kv, t0 = it.t0, L = it.L, gs = it.gs;
+      const int h = it.h, s = it.s, kv = it.kv, t0 = it.t0, L = it.L, gs = it.gs;
       const int ntq = q ? it.nt1 : it.nt0;
       const uint64_t word = q ? it.w1 : it.w0;
       const int row0 = (it.qt0 + q) * BM;
       const int my_row = row0 + tr;
       const float q_sc = __ldg(p.q_scale + static_cast<size_t>(h) * p.total_qtiles + it.cq + it.qt0 + q);
       const float* ks = p.k_scale + static_cast<size_t>(kv) * p.total_ktiles + it.ck;
+      (void)s;
       SoftmaxCtx cx;
       cx.p = &p;
       cx.bars = bars;
       cx.abort_flag = abort_flag;
       cx.tmo = tmo;
-      cx.tb = tmem + lane_base + S::col_b(q, 0);
+      cx.ts = tmem + lane_base + S::col_s(q);
       cx.to = tmem + lane_base + S::col_o(q);
+      cx.tp0 = tmem + lane_base + S::col_p(q, 0);
       cx.q = q;
       cx.L = L;
       cx.row0 = row0;
@@ -793,7 +786,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       st.l = 0.f;
       st.k_sc_next = __ldg(ks);
       st.n_s = n_s;
-      st.n_pvl = n_pvl;
+      st.n_p = n_p;
       // Key tiles before the first one that needs the legality mask (the
       // diagonal tiles of a causal row, a sequence's ragged last tile) run the
       // lean body, the rest the masked one; a debug run takes the body with
@@ -821,7 +814,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           break;
         }
       n_s = st.n_s;
-      if (ntq >= 2) ++n_pvl;
+      n_p = st.n_p;
       const float m = st.m, l = st.l;
       // o_final's next phase needs o_free from this epilogue
       if (!ok || !wait_bar_warp(&bars->o_final[q], n_items & 1, abort_flag, tmo)) {
