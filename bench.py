@@ -35,7 +35,7 @@ METRIC = "attention prefill tok/s at 4k b8 (3B GQA shape); % of mixed tensor roo
 UNIT = "tok/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-INT8_OVER_F16 = 4.5 / 2.25  # nominal dense INT8 : FP16 tensor rate on B200
+INT8_OVER_F16 = 4.5 / 2.25  # nominal dense INT8 : FP16 tensor rate on B200 (context only)
 
 
 # ----------------------------------------------------------------- helpers ---
@@ -168,6 +168,20 @@ def max_over_ranks(values, device=None):
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(x) for x in t.cpu()]
+
+
+def low_over_f16(low="int8"):
+    """Measured dense rate ratio of the low-precision MMA form to the FP16 one
+    on this GPU: tcgen05.mma M128 N256 issued back to back on every SM
+    (tilemix_mma_rate), kind::i8 (or kind::f8f6f4) with K = 32 against
+    kind::f16 with K = 16, from the SM cycles per MMA.  Returns the ratio and
+    the two measurements."""
+    import tile_routed_mixed_b200 as tm
+    f16 = tm.mma_rate("f16", 256, iters=2048)
+    lo = tm.mma_rate("i8" if low == "int8" else "f8", 256, iters=2048)
+    per_cycle_f16 = 2 * 128 * 256 * 16 / f16["cycles_per_mma"]
+    per_cycle_lo = 2 * 128 * 256 * 32 / lo["cycles_per_mma"]
+    return per_cycle_lo / per_cycle_f16, f16, lo
 
 
 def whole_job_tokens(tokens_per_rank, world):
@@ -415,7 +429,8 @@ def run_gpu(args):
     f16, i8, nbytes = algorithmic_work(lengths, hq, hk, d, masks, g, causal)
     pk = peaks()
     p16 = pk["bf16_tflops"] * 1e12
-    p8 = p16 * INT8_OVER_F16
+    ratio, r16, rlo = low_over_f16(args.low)
+    p8 = p16 * ratio
     t_tensor = f16 / p16 + i8 / p8
     t_mem = nbytes / (pk["hbm_gbs"] * 1e9)
     bound = "tensor" if t_tensor >= t_mem else "hbm"
@@ -451,6 +466,12 @@ def run_gpu(args):
             "mixed_roof_ms": 1e3 * max(t_tensor, t_mem),
             "tflops_raw": (f16 + i8) / t_k / 1e12,
             "int8_share_of_legal_groups": float(int8.sum() / legal.sum()),
+            "low_over_fp16_rate": {
+                "measured": ratio, "nominal": INT8_OVER_F16,
+                "how": "tcgen05.mma M128 N256 back to back on every SM: %s %.1f cycles per MMA "
+                       "(K 32), kind::f16 %.1f (K 16)" % (
+                           "kind::i8" if args.low == "int8" else "kind::f8f6f4",
+                           rlo["cycles_per_mma"], r16["cycles_per_mma"])},
         },
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": int(q.nbytes + k.nbytes + v.nbytes),
@@ -989,6 +1010,34 @@ def run_mad(args):
                       "rows_sampled": int(rows.shape[0]), "mad": out}), flush=True)
 
 
+def run_mma(args):
+    """Dense rate of each MMA form the fused kernel issues (tcgen05.mma, M128,
+    issued back to back by one thread per CTA on every SM; tilemix_mma_rate):
+    SM cycles per MMA and TFLOP/s (TOP/s) at the clock the run saw, and the
+    INT8 : FP16 and FP8 : FP16 rate ratios the mixed roofline uses."""
+    import torch
+    import tile_routed_mixed_b200 as tm
+    torch.cuda.init()
+    uuid = str(torch.cuda.get_device_properties(0).uuid)
+    smi = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    smi.start()
+    rows = []
+    for form, k in (("f16", 16), ("i8", 32), ("f8", 32), ("f16_tmem_a", 16)):
+        for n in (64, 128, 256):
+            r = tm.mma_rate(form, n, iters=4096)
+            r["k"] = k
+            r["macs_per_cycle"] = 128 * n * k / r["cycles_per_mma"]
+            rows.append(r)
+    clocks = smi.stop()
+    by = {(r["form"], r["n"]): r for r in rows}
+    ratio = lambda a, b: by[(a, 256)]["macs_per_cycle"] / by[(b, 256)]["macs_per_cycle"]
+    line = {"metric": "tcgen05.mma dense rate of the fused kernel's MMA forms (M128, every SM)",
+            "value": ratio("i8", "f16"), "unit": "INT8 : FP16 rate (N256)",
+            "fp8_over_fp16": ratio("f8", "f16"), "forms": rows, "clocks": clocks,
+            "n_gpus": 1, "data": "synthetic"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1001,10 +1050,11 @@ def main():
     ap.add_argument("--low", choices=["int8", "fp8"], default="int8",
                     help="low-precision path of bit-1 tiles in the prefill bench (fp8 = e4m3)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["prefill", "decode", "route", "mass", "mad"],
+    ap.add_argument("--path", choices=["prefill", "decode", "route", "mass", "mad", "mma"],
                     default="prefill",
                     help="prefill (the headline metric), the decode step with the INT8 K "
-                         "cache, or pooled-score adaptive routing")
+                         "cache, pooled-score adaptive routing, the importance-mass probe, "
+                         "the deviation table, or the tcgen05 rate of the kernel's MMA forms")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -1016,6 +1066,8 @@ def main():
         run_mass(args)
     elif args.path == "mad":
         run_mad(args)
+    elif args.path == "mma":
+        run_mma(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
