@@ -76,6 +76,24 @@ def test_routing_builder_bit_exact_vs_oracle(geom, template):
             assert np.array_equal(legal, lo) and np.array_equal(int8, io)
 
 
+@pytest.mark.parametrize("fname,template,percent,L", [
+    ("sptrans_l640_p75.txt", "sptrans", 75, 640),
+    ("sptrans_l1024_p50.txt", "sptrans", 50, 1024),
+    ("aligned_sparse_l1024_p25.txt", "aligned_sparse", 25, 1024),
+    ("aligned_sparse_l1024_p30.txt", "aligned_sparse", 30, 1024),
+    ("row_random_l640_p50_seed0.txt", "row_random", 50, 640),
+    ("bigbird_l640_p50_seed0.txt", "bigbird", 50, 640),
+    ("band_tiny_l256.txt", "band", 50, 256),
+], ids=lambda x: str(x))
+def test_routing_builder_hand_golden(fname, template, percent, L):
+    # the library's host builder against the hand-derived words directly
+    with open(os.path.join(ROOT, "tests", "golden", fname)) as f:
+        want = [int(x, 16) for x in f if x.strip() and not x.startswith("#")]
+    m, _, _ = tm.tilemix_build_routing(template, percent, 0, synth.cu_seqlens_of([L]), 1, [1],
+                                       True)
+    assert [int(x) for x in m[:, 0]] == want
+
+
 def test_routing_builder_rejects_bad_arguments():
     cu = synth.cu_seqlens_of([8192])
     with pytest.raises(tm.TileMixError) as e:

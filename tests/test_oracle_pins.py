@@ -168,6 +168,36 @@ def test_band_tiny_golden():
     assert list(legal) == [6] and list(int8) == [3]
 
 
+# Hand-derived routing words (derivation in each file's header): SpTrans's
+# stride and tail, the proportional quota's remainder rule with ties, and the
+# seeded Row-Random / BigBird shuffles at seed 0.
+TEMPLATE_GOLDENS = [
+    ("sptrans_l640_p75.txt", "sptrans", 75, 640),
+    ("sptrans_l1024_p50.txt", "sptrans", 50, 1024),
+    ("aligned_sparse_l1024_p25.txt", "aligned_sparse", 25, 1024),
+    ("aligned_sparse_l1024_p30.txt", "aligned_sparse", 30, 1024),
+    ("row_random_l640_p50_seed0.txt", "row_random", 50, 640),
+    ("bigbird_l640_p50_seed0.txt", "bigbird", 50, 640),
+]
+
+
+@pytest.mark.parametrize("fname,template,percent,L", TEMPLATE_GOLDENS, ids=lambda x: str(x))
+def test_template_hand_golden(fname, template, percent, L):
+    want = [int(x, 16) for x in _golden_lines(fname)]
+    m, legal, int8 = oracle.build_routing(template, percent, 0, [L], 2, [1], True)
+    assert [int(x) for x in m[:, 0]] == want
+    assert [int(x) for x in m[:, 1]] == want
+    assert int(legal[0]) == sum(2 * qt + 2 for qt in range(L // 128))
+    assert int(int8[0]) == sum(bin(w).count("1") for w in want)
+
+
+def test_row_streams_are_the_splitmix64_sequence():
+    # row qt's stream state draw(0, qt + 1) is the (qt+1)-th splitmix64 output
+    # from state 0, the values of splitmix64_state0.txt
+    want = [int(x, 16) for x in _golden_lines("splitmix64_state0.txt")]
+    assert [oracle.routing._draw(0, qt + 1) for qt in range(3)] == want
+
+
 def _workload_geometry(name):
     w = synth.WORKLOADS[name]
     lengths = synth.workload_lengths(name)
