@@ -40,13 +40,17 @@ INT8_OVER_F16 = 4.5 / 2.25  # nominal dense INT8 : FP16 tensor rate on B200 (con
 
 # ----------------------------------------------------------------- helpers ---
 
-def workload(name, template=None, percent=None):
+def workload(name, template=None, percent=None, seqs=None):
+    """A configuration's sizes; `seqs` keeps only its first sequences (a
+    smaller case of the same shapes, for profiler captures)."""
     w = dict(synth.WORKLOADS[name])
     if template:
         w["template"] = template
     if percent is not None:
         w["percent"] = int(percent)
     lengths = synth.workload_lengths(name)
+    if seqs:
+        lengths = lengths[:int(seqs)]
     if w["g"] == "auto":
         g = [max(1, math.ceil(math.ceil(L / 64) / 64)) for L in lengths]
     else:
@@ -279,7 +283,7 @@ def run_reference(args):
         # alone here, so give the oracle every core (before any OpenMP
         # runtime loads)
         os.environ["OMP_NUM_THREADS"] = str(affinity_cores())
-    w, lengths, g = workload(args.workload, args.template, args.percent)
+    w, lengths, g = workload(args.workload, args.template, args.percent, args.seqs)
     hq, hk, d, causal = w["hq"], w["hk"], w["d"], w["causal"]
     T = sum(lengths)
     q, k, v = synth.make_qkv(0, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
@@ -341,7 +345,7 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    w, lengths, g = workload(args.workload, args.template, args.percent)
+    w, lengths, g = workload(args.workload, args.template, args.percent, args.seqs)
     hq, hk, d, causal = w["hq"], w["hk"], w["d"], w["causal"]
     T = sum(lengths)
     q, k, v = synth.make_qkv(rank, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
@@ -528,7 +532,7 @@ def run_decode(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference" and rank != 0:
         return
-    w, lengths, g = workload(args.workload, args.template, args.percent)
+    w, lengths, g = workload(args.workload, args.template, args.percent, args.seqs)
     hq, hk, d = w["hq"], w["hk"], w["d"]
     if args.impl != "reference":
         import torch
@@ -690,7 +694,7 @@ def run_route(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference" and rank != 0:
         return
-    w, lengths, g = workload(args.workload, args.template, args.percent)
+    w, lengths, g = workload(args.workload, args.template, args.percent, args.seqs)
     hq, hk, d = w["hq"], w["hk"], w["d"]
     T = sum(lengths)
     q, k, _ = synth.make_qkv(rank, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
@@ -833,7 +837,7 @@ def run_mass(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference" and rank != 0:
         return
-    w, lengths, g = workload(args.workload, args.template, args.percent)
+    w, lengths, g = workload(args.workload, args.template, args.percent, args.seqs)
     hq, hk, d, causal = w["hq"], w["hk"], w["d"], w["causal"]
     T = sum(lengths)
     q, k, _ = synth.make_qkv(rank, T, hq, hk, d, outliers=w["outliers"], lowrank=w["lowrank"])
@@ -984,7 +988,7 @@ def run_mad(args):
     from oracle import fp8 as of8
     from tests import gpu_cases as gc
 
-    w, lengths, g = workload(args.workload, args.template, args.percent)
+    w, lengths, g = workload(args.workload, args.template, args.percent, args.seqs)
     case = gc.Case.workload(args.workload)
     q, k, v = case.inputs()
     rows = gc.sample_rows(case.lengths, case.hq, seed=3, per_head_random=16,
@@ -1050,6 +1054,8 @@ def main():
     ap.add_argument("--low", choices=["int8", "fp8"], default="int8",
                     help="low-precision path of bit-1 tiles in the prefill bench (fp8 = e4m3)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqs", type=int, default=None,
+                    help="keep only the first N sequences of the workload (profiler captures)")
     ap.add_argument("--path", choices=["prefill", "decode", "route", "mass", "mad", "mma"],
                     default="prefill",
                     help="prefill (the headline metric), the decode step with the INT8 K "
