@@ -6,7 +6,7 @@ link or run anything in this package.  The library's product path never does:
 it fails loudly when its CUDA extension is missing instead of falling back here.
 
 The oracle is plain and slow on purpose: numpy for block quantisation
-(``quant.py``), pure Python for the routing templates (``routing.py``, with its
+(``quant.py``, INT8 and INT4 codes), pure Python for the routing templates (``routing.py``, with its
 own splitmix64), and plain C in fp64 / int64 for the attention rows
 (``attention_oracle.c``, OpenMP over rows, no blocking); the decode step
 (``decode.py``) composes those; ``adaptive.py`` restates the pooled-score
@@ -34,7 +34,7 @@ output value comes from the pages.
 from . import adaptive, fp8, mass
 from .attention import all_rows, attention_rows, build, half_to_double, int_scores
 from .decode import decode_rows, quantize_rows
-from .quant import quantize_blocks, quantize_k, quantize_q
+from .quant import quantize_blocks, quantize_k, quantize_k_int4, quantize_q, quantize_q_int4
 from .routing import (BLOCK_M, BLOCK_N, MAX_GROUPS, TEMPLATES, auto_g, build_routing,
                       fp16_groups, int8_target, last_legal_tile, legal_groups, n_ktiles,
                       n_qtiles, tile_offsets)
@@ -44,5 +44,5 @@ __all__ = [
     "build", "build_routing", "decode_rows", "fp16_groups", "half_to_double", "int8_target",
     "int_scores",
     "last_legal_tile", "legal_groups", "n_ktiles", "n_qtiles", "quantize_blocks",
-    "quantize_k", "quantize_q", "tile_offsets",
+    "quantize_k", "quantize_k_int4", "quantize_q", "quantize_q_int4", "tile_offsets",
 ]

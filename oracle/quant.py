@@ -11,6 +11,11 @@ and one head (it never crosses a sequence; a short tail block uses its valid
 rows only).  a = max |x| over the block (x is the fp16 value, exact in fp32);
 s = fp32(a / 127) with IEEE division; code = clamp(round_half_even(fp32(x / s)),
 -127, 127); a block with a == 0 has s = 0 and all codes 0.
+
+INT4 codes (the 4-bit format the same pages name as an open alternative to
+INT8: agihunt, limitations paragraph; 59188saintaubert.com explainer, closing
+section): the same blocks and rule with 7 in place of 127, s = fp32(a / 7) and
+codes in [-7, 7] (kept one per byte).
 """
 from __future__ import annotations
 
@@ -19,8 +24,9 @@ import numpy as np
 from .routing import BLOCK_M, BLOCK_N
 
 
-def quantize_blocks(x16: np.ndarray, lengths, block: int):
-    """x16 [T, H, d] float16 -> (codes int8 [T, H, d], scales float32 [H, total_blocks])."""
+def quantize_blocks(x16: np.ndarray, lengths, block: int, qmax: int = 127):
+    """x16 [T, H, d] float16 -> (codes int8 [T, H, d], scales float32 [H, total_blocks]);
+    qmax = 127 for INT8 codes, 7 for INT4 codes."""
     if x16.dtype != np.float16 or x16.ndim != 3:
         raise ValueError("expected float16 [T, H, d]")
     T, H, d = x16.shape
@@ -37,9 +43,9 @@ def quantize_blocks(x16: np.ndarray, lengths, block: int):
                 r1 = min(t0 + L, r0 + block)
                 blk = x16[r0:r1].astype(np.float32)             # exact
                 a = np.abs(blk).max(axis=(0, 2))                  # [H]
-                s = (a / np.float32(127.0)).astype(np.float32)    # IEEE fp32 division
+                s = (a / np.float32(qmax)).astype(np.float32)     # IEEE fp32 division
                 q = blk / s[None, :, None]                        # IEEE fp32 division
-                c = np.clip(np.rint(q), -127, 127)                # half-to-even
+                c = np.clip(np.rint(q), -qmax, qmax)              # half-to-even
                 c = np.where((a == 0)[None, :, None], 0, c)
                 c = np.nan_to_num(c, nan=0.0)
                 codes[r0:r1] = c.astype(np.int8)
@@ -55,3 +61,11 @@ def quantize_q(q16, lengths):
 
 def quantize_k(k16, lengths):
     return quantize_blocks(k16, lengths, BLOCK_N)
+
+
+def quantize_q_int4(q16, lengths):
+    return quantize_blocks(q16, lengths, BLOCK_M, qmax=7)
+
+
+def quantize_k_int4(k16, lengths):
+    return quantize_blocks(k16, lengths, BLOCK_N, qmax=7)

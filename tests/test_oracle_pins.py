@@ -142,6 +142,75 @@ def test_quantiser_error_bound_random():
             col += nb
 
 
+def test_int4_quantiser_hand_cases():
+    for line in _golden_lines("quant_int4_hand_cases.txt"):
+        vals, codes = line.split(";")
+        vals = np.array([float(x) for x in vals.split()], dtype=np.float64)
+        codes = np.array([int(x) for x in codes.split()], dtype=np.int64)
+        x = np.zeros((64, 1, vals.size), dtype=np.float16)
+        x[0, 0] = vals
+        x[1, 0, 0] = 7.0   # absmax of the block is 7 -> scale 1
+        c, s = oracle.quantize_k_int4(x, [64])
+        assert s[0, 0] == np.float32(1.0)
+        assert np.array_equal(c[0, 0].astype(np.int64), codes)
+
+
+def test_int4_quantiser_bounds_zero_blocks_and_tails():
+    x = np.zeros((64, 2, 8), dtype=np.float16)
+    x[:, 1] = -3.0
+    c, s = oracle.quantize_k_int4(x, [64])
+    assert s[0, 0] == 0 and not c[:, 0].any()
+    assert s[1, 0] == np.float32(3.0) / np.float32(7.0) and (c[:, 1] == -7).all()
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((300, 3, 64)) * rng.uniform(0.01, 50, (1, 3, 1))).astype(np.float16)
+    lengths = [130, 170]
+    for block, fn in ((64, oracle.quantize_k_int4), (128, oracle.quantize_q_int4)):
+        c, s = fn(x, lengths)
+        t0, col = 0, 0
+        for L in lengths:
+            nb = -(-L // block)
+            for b in range(nb):
+                r0, r1 = t0 + b * block, min(t0 + L, t0 + (b + 1) * block)
+                for h in range(3):
+                    blk = x[r0:r1, h].astype(np.float64)
+                    cc = c[r0:r1, h].astype(np.float64)
+                    sc = float(s[h, col + b])
+                    # the block's largest |x| maps to 7; every code within +-7
+                    assert np.abs(cc).max() == 7 and np.all(np.abs(cc) <= 7)
+                    assert sc == float(np.float32(np.abs(blk).max()) / np.float32(7.0))
+                    # |code * s - x| <= s / 2 up to fp32 rounding of x / s
+                    assert np.all(np.abs(cc * sc - blk) <= sc * (0.5 + 1e-5))
+            t0 += L
+            col += nb
+
+
+def test_int4_codes_through_the_routed_attention():
+    # INT4 codes take the INT8 path's arithmetic (exact integer dots times the
+    # two block scales): the oracle fed INT4 codes equals the per-key brute
+    # force on the same codes, and all-INT4 words deviate from all-FP16 more
+    # than all-INT8 words do
+    lengths = [100, 300, 64]
+    hq, hk, d = 4, 2, 64
+    q, k, v, _, _, _, _ = _inputs(lengths, hq, hk, d, seed=4)
+    q4, qs4 = oracle.quantize_q_int4(q, lengths)
+    k4, ks4 = oracle.quantize_k_int4(k, lengths)
+    assert np.abs(q4).max() <= 7 and np.abs(k4).max() <= 7
+    inp4 = (q, k, v, q4, qs4, k4, ks4)
+    tm = sum(oracle.n_qtiles(L) for L in lengths)
+    rng = np.random.default_rng(3)
+    masks = rng.integers(0, 2 ** 63, size=(tm, hk), dtype=np.uint64) * np.uint64(2) + \
+        rng.integers(0, 2, size=(tm, hk), dtype=np.uint64)
+    gs = [1] * len(lengths)
+    O, lse = _run(inp4, masks, gs, lengths, True)
+    Or, lr = bf.routed_attention(*inp4, masks, gs, lengths, True)
+    assert np.abs(O - Or).max() < 1e-12 and np.abs(lse - lr).max() < 1e-12
+    ones = _words(lengths, hk, (1 << 64) - 1)
+    base, _ = _run(inp4, _words(lengths, hk, 0), gs, lengths, True)
+    dev4 = np.abs(_run(inp4, ones, gs, lengths, True)[0] - base).mean()
+    dev8 = np.abs(_run(_inputs(lengths, hq, hk, d, seed=4), ones, gs, lengths, True)[0] - base).mean()
+    assert dev4 > 4 * dev8
+
+
 # --------------------------------------------------------------------------
 # routing pins
 # --------------------------------------------------------------------------
