@@ -182,7 +182,7 @@ def low_over_f16(low="int8"):
     the two measurements."""
     import tile_routed_mixed_b200 as tm
     f16 = tm.mma_rate("f16", 256, iters=2048)
-    lo = tm.mma_rate("i8" if low == "int8" else "f8", 256, iters=2048)
+    lo = tm.mma_rate("f8" if low == "fp8" else "i8", 256, iters=2048)  # INT4 codes: kind::i8
     per_cycle_f16 = 2 * 128 * 256 * 16 / f16["cycles_per_mma"]
     per_cycle_lo = 2 * 128 * 256 * 32 / lo["cycles_per_mma"]
     return per_cycle_lo / per_cycle_f16, f16, lo
@@ -456,7 +456,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16+i8" if args.low == "int8" else "f16+e4m3",
+        "dtype": {"int8": "f16+i8", "fp8": "f16+e4m3", "int4": "f16+i4(in i8)"}[args.low],
         "data": "synthetic",
         "config": bench_config(args, w, lengths, g),
         "roofline": {
@@ -474,7 +474,7 @@ def run_gpu(args):
                 "measured": ratio, "nominal": INT8_OVER_F16,
                 "how": "tcgen05.mma M128 N256 back to back on every SM: %s %.1f cycles per MMA "
                        "(K 32), kind::f16 %.1f (K 16)" % (
-                           "kind::i8" if args.low == "int8" else "kind::f8f6f4",
+                           "kind::f8f6f4" if args.low == "fp8" else "kind::i8",
                            rlo["cycles_per_mma"], r16["cycles_per_mma"])},
         },
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
@@ -1000,7 +1000,7 @@ def run_mad(args):
                                    case.causal, rows=rows)
     qd, kd, vd = (torch.from_numpy(x).cuda() for x in (q, k, v))
     out = {}
-    for low in ("int8", "fp8"):
+    for low in ("int8", "fp8", "int4"):
         for pct in (0, 10, 25, 50, 75, 100):
             masks = oracle.build_routing(case.template, pct, case.routing_seed, case.lengths,
                                          case.hk, case.g, case.causal)[0]
@@ -1051,7 +1051,7 @@ def main():
     ap.add_argument("--workload", default="llama3b_4k_b8", choices=list(synth.WORKLOADS))
     ap.add_argument("--template", default=None)
     ap.add_argument("--percent", type=int, default=None)
-    ap.add_argument("--low", choices=["int8", "fp8"], default="int8",
+    ap.add_argument("--low", choices=["int8", "fp8", "int4"], default="int8",
                     help="low-precision path of bit-1 tiles in the prefill bench (fp8 = e4m3)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", type=int, default=None,

@@ -159,6 +159,19 @@ int tilemix_quantize_qk_fp8(const void* q_f16, const void* k_f16, const int32_t*
                             int d, int8_t* q_codes, float* q_scale, int8_t* k_codes,
                             float* k_scale, void* stream);
 
+/* INT4 low path (the 4-bit integer format the TileMix pages name as an open
+ * alternative to INT8: agihunt summary, limitations paragraph; explainer,
+ * closing section): the blocks and rounding of tilemix_quantize_qk with 7 in
+ * place of 127, s = fp32(a / 7), code = rne(fp32(x / s)) in [-7, 7], one code
+ * per int8 element (sm_100a has no 4-bit integer tensor-core kind: the codes
+ * take the INT8 MMA, whose int32 dots stay exact).  Arguments, layouts and
+ * errors as tilemix_quantize_qk. */
+int tilemix_quantize_qk_int4(const void* q_f16, const void* k_f16, const int32_t* cu_seqlens_d,
+                             const int32_t* cu_qtiles_d, const int32_t* cu_ktiles_d, int nseq,
+                             int total_tokens, int total_qtiles, int total_ktiles, int hq, int hk,
+                             int d, int8_t* q_codes, float* q_scale, int8_t* k_codes,
+                             float* k_scale, void* stream);
+
 typedef struct tilemix_prefill_args {
   const void* q;          /* device fp16 [total_tokens][hq][d], 16-byte aligned */
   const void* k;          /* device fp16 [total_tokens][hk][d], 16-byte aligned */
@@ -198,7 +211,9 @@ typedef struct tilemix_prefill_args {
                                   (the pages' method, default), 1 = FP8 e4m3 (see
                                   tilemix_quantize_qk_fp8; k_i8 / k_scale, when given,
                                   then hold e4m3 codes and their scales; no debug
-                                  INT32 dump) */
+                                  INT32 dump), 2 = INT4 codes on the INT8 MMA (see
+                                  tilemix_quantize_qk_int4; k_i8 / k_scale, when
+                                  given, hold INT4 codes and their scales) */
 } tilemix_prefill_args;
 
 /* Bytes of device workspace tilemix_prefill_fwd needs for these arguments

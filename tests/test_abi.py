@@ -141,7 +141,8 @@ def test_prefill_argument_checks_are_synchronous():
     assert n.value == 131072 + 256 + 256
     cases = [
         (dict(d=96), tm.ERR_UNSUPPORTED),
-        (dict(low_format=2), tm.ERR_INVALID_ARG),
+        (dict(low_format=3), tm.ERR_INVALID_ARG),
+        (dict(low_format=-1), tm.ERR_INVALID_ARG),
         (dict(low_format=1, debug_int32_scores=4096), tm.ERR_UNSUPPORTED),
         (dict(hq=3, hk=2), tm.ERR_INVALID_ARG),
         (dict(hk=0), tm.ERR_INVALID_ARG),

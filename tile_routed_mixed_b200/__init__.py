@@ -53,7 +53,7 @@ class PrefillArgs(ctypes.Structure):
     ]
 
 
-LOW_FORMATS = {"int8": 0, "fp8": 1}
+LOW_FORMATS = {"int8": 0, "fp8": 1, "int4": 2}
 
 
 class PrefillHostArgs(ctypes.Structure):
@@ -142,6 +142,8 @@ def lib():
         L.tilemix_quantize_qk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P]
         L.tilemix_quantize_qk_fp8.restype = I
         L.tilemix_quantize_qk_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P]
+        L.tilemix_quantize_qk_int4.restype = I
+        L.tilemix_quantize_qk_int4.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P]
         L.tilemix_workspace_size.restype = I
         L.tilemix_workspace_size.argtypes = [ctypes.POINTER(PrefillArgs),
                                              ctypes.POINTER(ctypes.c_size_t)]
@@ -275,6 +277,18 @@ def tilemix_quantize_qk_fp8(q, k, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_
                                          int(d), _ptr(q_codes), _ptr(q_scale), _ptr(k_codes),
                                          _ptr(k_scale), _stream_handle(stream)),
            "tilemix_quantize_qk_fp8")
+
+
+def tilemix_quantize_qk_int4(q, k, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_tokens,
+                             total_qtiles, total_ktiles, hq, hk, d, q_codes, q_scale, k_codes,
+                             k_scale, stream=None):
+    """The INT4 low path's codes (in [-7, 7], one per int8 element) and scales."""
+    _check(lib().tilemix_quantize_qk_int4(_ptr(q), _ptr(k), _ptr(cu_seqlens), _ptr(cu_qtiles),
+                                          _ptr(cu_ktiles), int(nseq), int(total_tokens),
+                                          int(total_qtiles), int(total_ktiles), int(hq), int(hk),
+                                          int(d), _ptr(q_codes), _ptr(q_scale), _ptr(k_codes),
+                                          _ptr(k_scale), _stream_handle(stream)),
+           "tilemix_quantize_qk_int4")
 
 
 def make_args(q, k, v, o, cu_seqlens, cu_qtiles, cu_ktiles, nseq, total_tokens, total_qtiles,
@@ -498,7 +512,7 @@ from .decode import TileMixDecode  # noqa: E402  (convenience wrapper)
 __all__ = [
     "BLOCK_M", "BLOCK_N", "DecodeArgs", "MAX_GROUPS", "PrefillArgs", "RouteArgs", "TEMPLATES",
     "TileMixError", "route_pooled", "tilemix_route_pooled", "tilemix_route_workspace_size",
-    "LOW_FORMATS", "tilemix_quantize_qk_fp8",
+    "LOW_FORMATS", "tilemix_quantize_qk_fp8", "tilemix_quantize_qk_int4",
     "MassArgs", "mass_probe", "tilemix_mass_probe",
     "TileMixDecode", "TileMixPrefill", "lib", "make_args", "status_string", "tilemix_auto_g",
     "tilemix_build_routing", "tilemix_decode_fwd", "tilemix_decode_workspace_size",

@@ -100,7 +100,7 @@ int check_args(const tilemix_prefill_args* a) {
   if (a->causal != 0 && a->causal != 1) return TILEMIX_ERR_INVALID_ARG;
   if (!(a->softmax_scale >= 0.f) || std::isinf(a->softmax_scale)) return TILEMIX_ERR_INVALID_ARG;
   if ((a->k_i8 == nullptr) != (a->k_scale == nullptr)) return TILEMIX_ERR_INVALID_ARG;
-  if (a->low_format != 0 && a->low_format != 1) return TILEMIX_ERR_INVALID_ARG;
+  if (a->low_format < 0 || a->low_format > 2) return TILEMIX_ERR_INVALID_ARG;
   if (a->low_format == 1 && a->debug_int32_scores) return TILEMIX_ERR_UNSUPPORTED;
   if (a->nseq == 0 || a->total_tokens == 0) return TILEMIX_OK;  // nothing to do
   if (!a->q || !a->k || !a->v || !a->o || !a->cu_seqlens || !a->cu_qtiles || !a->cu_ktiles ||
@@ -119,7 +119,7 @@ int quantize_impl(const void* q_f16, const void* k_f16, const int32_t* cu_seqlen
                   const int32_t* cu_qtiles_d, const int32_t* cu_ktiles_d, int nseq,
                   int total_tokens, const tilemix::QuantRange& range, int total_qtiles,
                   int total_ktiles, int hq, int hk, int d, int8_t* q_i8, float* q_scale,
-                  int8_t* k_i8, float* k_scale, int* ticket, int fp8, void* stream) {
+                  int8_t* k_i8, float* k_scale, int* ticket, int fmt, void* stream) {
   if (d != 64 && d != 128) return TILEMIX_ERR_UNSUPPORTED;
   if (nseq < 0 || total_tokens < 0 || total_qtiles < 0 || total_ktiles < 0)
     return TILEMIX_ERR_INVALID_ARG;
@@ -138,7 +138,7 @@ int quantize_impl(const void* q_f16, const void* k_f16, const int32_t* cu_seqlen
   }
   if (tilemix::launch_quantize_qk(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq,
                                   range, total_qtiles, total_ktiles, hq, hk, d, q_i8, q_scale,
-                                  k_i8, k_scale, ticket, fp8, st) != cudaSuccess)
+                                  k_i8, k_scale, ticket, fmt, st) != cudaSuccess)
     return TILEMIX_ERR_CUDA;
   return TILEMIX_OK;
 }
@@ -209,7 +209,7 @@ int plan_prefill(const tilemix_prefill_args* a, PrefillPlan* pl) {
   p.causal = a->causal;
   const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.low_fp8 = a->low_format;
+  p.low_fp8 = a->low_format == 1;  // INT4 codes take the INT8 MMA path
   p.timeout_ns = wait_timeout_ns();
   return TILEMIX_OK;
 }
@@ -283,6 +283,17 @@ TILEMIX_API int tilemix_quantize_qk_fp8(const void* q_f16, const void* k_f16,
   return quantize_impl(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq, total_tokens,
                        {0, total_qtiles, 0, total_ktiles}, total_qtiles, total_ktiles, hq, hk, d,
                        q_codes, q_scale, k_codes, k_scale, nullptr, 1, stream);
+}
+
+TILEMIX_API int tilemix_quantize_qk_int4(const void* q_f16, const void* k_f16,
+                                        const int32_t* cu_seqlens_d, const int32_t* cu_qtiles_d,
+                                        const int32_t* cu_ktiles_d, int nseq, int total_tokens,
+                                        int total_qtiles, int total_ktiles, int hq, int hk, int d,
+                                        int8_t* q_codes, float* q_scale, int8_t* k_codes,
+                                        float* k_scale, void* stream) {
+  return quantize_impl(q_f16, k_f16, cu_seqlens_d, cu_qtiles_d, cu_ktiles_d, nseq, total_tokens,
+                       {0, total_qtiles, 0, total_ktiles}, total_qtiles, total_ktiles, hq, hk, d,
+                       q_codes, q_scale, k_codes, k_scale, nullptr, 2, stream);
 }
 
 TILEMIX_API int tilemix_workspace_size(const tilemix_prefill_args* args, size_t* bytes) {

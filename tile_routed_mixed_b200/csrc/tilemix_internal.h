@@ -42,7 +42,8 @@ struct PrefillParams {
   int hq, hk, group;      // group = hq / hk
   int causal;
   float scale_log2;       // softmax scale * log2(e)
-  int low_fp8;            // low-precision tiles: 0 INT8 (kind::i8), 1 FP8 e4m3 (kind::f8f6f4)
+  int low_fp8;            // low-precision tiles: 0 integer codes (INT8 or INT4, kind::i8),
+                          // 1 FP8 e4m3 (kind::f8f6f4)
   unsigned long long timeout_ns;
 };
 
@@ -135,7 +136,7 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
                        const QuantRange& range, int total_qtiles, int total_ktiles, int hq,
                        int hk, int d, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
-                       int* ticket, int fp8, cudaStream_t stream);
+                       int* ticket, int fmt, cudaStream_t stream);  // fmt: 0 INT8, 1 FP8, 2 INT4
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
 int read_and_clear_status(unsigned int* status, cudaStream_t stream);
 // Device address of the allocation-free entry point's scratch array in the

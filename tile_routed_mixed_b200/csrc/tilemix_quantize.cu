@@ -35,14 +35,17 @@ struct QuantSide {
   int tile0, ntiles, total_tiles, heads, block_rows;
 };
 
-// fp8 != 0: the FP8 low path's codes instead, e4m3(x / s) with s = a / 448
-// (round to nearest even, saturating; IEEE fp32 division for both).
+// fmt selects the codes: 0 INT8 (s = a / 127), 2 INT4 (s = a / 7, codes in
+// [-7, 7], one per byte; the same rounding), 1 the FP8 low path's e4m3(x / s)
+// with s = a / 448 (round to nearest even, saturating; IEEE fp32 division for
+// both).
 // Thread t takes the 16-byte chunks of rows t / C + j 256 / C (C chunks per
 // row), column t mod C, for j < kChunks.
 template <int D>
 __global__ void __launch_bounds__(kQuantThreads, D == 128 ? 4 : 5)
     quantize_qk_kernel(QuantSide qs, QuantSide ks, const int32_t* __restrict__ cu_seqlens,
-                       int nseq, int* ticket, int fp8) {
+                       int nseq, int* ticket, int fmt) {
+  const bool fp8 = fmt == 1;
   constexpr int kCprLog2 = D == 128 ? 4 : 3;                 // 16-byte chunks per row
   constexpr int kRowsPerPass = kQuantThreads >> kCprLog2;    // rows one pass covers
   constexpr int kChunks = TILEMIX_BLOCK_M / kRowsPerPass;    // passes over a Q block
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(kQuantThreads, D == 128 ? 4 : 5)
   float a = red[0];
 #pragma unroll
   for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
-  const float s = __fdiv_rn(a, fp8 ? 448.0f : 127.0f);
+  const float s = __fdiv_rn(a, fp8 ? 448.0f : fmt == 2 ? 7.0f : 127.0f);
   if (threadIdx.x == 0) scales[static_cast<size_t>(h) * total_tiles + tile] = s;
   const float r = a > 0.f ? __frcp_rn(s) : 0.f;
   if (fp8) {
@@ -135,7 +138,7 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
                        const int32_t* cu_qtiles, const int32_t* cu_ktiles, int nseq,
                        const QuantRange& range, int total_qtiles, int total_ktiles, int hq,
                        int hk, int d, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
-                       int* ticket, int fp8, cudaStream_t stream) {
+                       int* ticket, int fmt, cudaStream_t stream) {
   QuantSide qs{static_cast<const __half*>(q), cu_qtiles, q8, q_scale, range.qtile0,
                q ? range.nqtiles : 0, total_qtiles, hq, TILEMIX_BLOCK_M};
   QuantSide ks{static_cast<const __half*>(k), cu_ktiles, k8, k_scale, range.ktile0,
@@ -147,10 +150,10 @@ int launch_quantize_qk(const void* q, const void* k, const int32_t* cu_seqlens,
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (d == 128)
     quantize_qk_kernel<128><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        qs, ks, cu_seqlens, nseq, ticket, fp8);
+        qs, ks, cu_seqlens, nseq, ticket, fmt);
   else
     quantize_qk_kernel<64><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        qs, ks, cu_seqlens, nseq, ticket, fp8);
+        qs, ks, cu_seqlens, nseq, ticket, fmt);
   return static_cast<int>(cudaGetLastError());
 }
 

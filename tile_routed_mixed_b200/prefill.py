@@ -27,7 +27,7 @@ class TileMixPrefill:
         self.max_seqlen = max(self.lengths) if self.lengths else 0
         self.causal = bool(causal)
         self.softmax_scale = float(softmax_scale)
-        self.low = str(low)  # low-precision path of bit-1 tiles: "int8" or "fp8" (e4m3)
+        self.low = str(low)  # low-precision path of bit-1 tiles: "int8", "fp8" (e4m3) or "int4"
         self.device = torch.device(device)
         masks = np.ascontiguousarray(masks, dtype=np.uint64)
         if masks.shape != (self.total_qtiles, self.hk):
