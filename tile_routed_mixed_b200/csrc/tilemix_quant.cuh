@@ -16,8 +16,7 @@ namespace tilemix {
 // round-to-nearest-even of the addition is rne of y, and the integer n sits
 // in the low mantissa bits: the sum's bit pattern is 0x4B400000 + n, whose low
 // byte is the two's-complement byte of n).  No clamp is needed: |f| <= a and
-// s = fl(a / qmax) give |y| < qmax + 0.0001, so rne(y) already lies in
-// [-qmax, qmax] (qmax = 127 for INT8 codes, 7 for INT4 codes).
+// s = fl(a / 127) give |y| < 127.0001, so rne(y) already lies in [-127, 127].
 constexpr float kRoundShift = 12582912.0f;  // 1.5 * 2^23
 constexpr float kBandEdge = 0.5f - 0x1p-12f;
 

@@ -36,8 +36,9 @@ struct QuantSide {
 };
 
 // fmt selects the codes: 0 INT8 (s = a / 127), 2 INT4 (s = a / 7, codes in
-// [-7, 7], one per byte; the same rounding), 1 the FP8 low path's e4m3(x / s)
-// with s = a / 448 (round to nearest even, saturating; IEEE fp32 division for
+// [-7, 7], one per byte; the same rounding, whose no-clamp argument holds with
+// 7 for 127: |x / s| < 7.0001), 1 the FP8 low path's e4m3(x / s) with
+// s = a / 448 (round to nearest even, saturating; IEEE fp32 division for
 // both).
 // Thread t takes the 16-byte chunks of rows t / C + j 256 / C (C chunks per
 // row), column t mod C, for j < kChunks.
