@@ -99,3 +99,11 @@ def test_fp8_and_int8_paths_differ_on_the_same_words():
         qd, kd, vd = (torch.from_numpy(x).cuda() for x in (q, k, v))
         outs.append(pf(qd, kd, vd).cpu().numpy().astype(np.float64))
     assert np.max(np.abs(outs[0] - outs[1])) > 1e-3
+
+
+def test_fp8_zero_length_sequences_and_custom_head_map():
+    # the FP8 flag with empty sequences in a packed batch and a
+    # non-contiguous head map
+    case = gc.Case([0, 300, 0, 129, 0], 4, 2, 128, template="bigbird", percent=50,
+                   kv_map=np.array([1, 0, 1, 0], dtype=np.int32), outliers=4, seed=46)
+    _prefill_fp8(case)

@@ -155,3 +155,39 @@ def test_int4_and_int8_paths_differ_on_the_same_words():
         qd, kd, vd = (torch.from_numpy(x).cuda() for x in (q, k, v))
         outs.append(pf(qd, kd, vd).cpu().numpy().astype(np.float64))
     assert np.max(np.abs(outs[0] - outs[1])) > 1e-3
+
+
+def test_int4_zero_length_sequences_custom_head_map_and_host_call():
+    # the INT4 flag through the remaining entry shapes: empty sequences in a
+    # packed batch, a non-contiguous head map, and the host-buffer call in
+    # runs of whole sequences (bit-equal to the device call)
+    import tile_routed_mixed_b200 as tm
+    kv_map = np.array([1, 0, 1, 0], dtype=np.int32)
+    case = gc.Case([0, 300, 0, 129, 0, 77], 4, 2, 128, template="sptrans", percent=75,
+                   kv_map=kv_map, outliers=4, seed=56)
+    q, k, v = case.inputs()
+    masks = case.masks()
+    pf = tm.TileMixPrefill(case.lengths, 4, 2, 128, masks, case.g, kv_head_of_q=kv_map,
+                           low="int4")
+    qd, kd, vd = (torch.from_numpy(x).cuda() for x in (q, k, v))
+    od = torch.full_like(qd, float("nan"))
+    pf(qd, kd, vd, od)
+    torch.cuda.synchronize()
+    assert tm.tilemix_get_error() == tm.OK
+    dev = od.cpu().numpy()
+    rows = oracle.all_rows(case.lengths, case.hq)
+    q4, qs = oracle.quantize_q_int4(q, case.lengths)
+    k4, ks = oracle.quantize_k_int4(k, case.lengths)
+    want, _ = oracle.attention_rows(q, k, v, q4, qs, k4, ks, masks, case.g, case.lengths,
+                                    case.causal, kv_map=kv_map, rows=rows)
+    mx, mn = gc.errors(gc.gather(case, dev, rows), want)
+    assert mx <= gc.MAX_ABS and mn <= gc.MEAN_ABS, (mx, mn)
+    qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    for chunks in (1, 4):
+        oh = torch.full(q.shape, float("nan"), dtype=torch.float16).pin_memory()
+        qd2, kd2, vd2 = (torch.empty(x.shape, dtype=torch.float16, device="cuda") for x in (q, k, v))
+        od2 = torch.empty(q.shape, dtype=torch.float16, device="cuda")
+        pf.from_host(qh, kh, vh, oh, qd2, kd2, vd2, od2, chunks=chunks)
+        torch.cuda.current_stream().synchronize()
+        assert tm.tilemix_get_error() == tm.OK
+        assert np.array_equal(oh.numpy().view(np.uint16), dev.view(np.uint16))
