@@ -461,7 +461,8 @@ def run_gpu(args):
         "config": bench_config(args, w, lengths, g),
         "roofline": {
             "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": kernel_traffic(args.workload),
+            "frac": achieved / peak,
+            "traffic": kernel_traffic(args.workload) if not args.seqs else None,
             "traffic_unit": "bytes per launch (ncu)",
             "kernel": "prefill_fwd_kernel<128>",
             "kernel_ms": kern_ms,
@@ -654,7 +655,8 @@ def run_decode(args):
         "data": "synthetic", "config": config,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"],
-                     "traffic": kernel_traffic(args.workload, "decode_attn_kernel<128>"),
+                     "traffic": (kernel_traffic(args.workload, "decode_attn_kernel<128>")
+                                 if not args.seqs else None),
                      "kernel": "decode_attn_kernel<128>", "kernel_ms": kern_ms,
                      "peak_kind": "copy bandwidth (%s)" % pk["source"],
                      "algorithmic_bytes": attn_bytes, "step_bytes": nbytes,
