@@ -527,6 +527,9 @@ def decode_bytes(lengths, hq, hk, d, masks, g):
     return total + requant + len(lengths) * hq * d * 2 * 2, attn
 
 
+DECODE_CACHES = 4  # copies of the decode cache the steps rotate over
+
+
 def run_decode(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -554,8 +557,9 @@ def run_decode(args):
     q_new = np.ascontiguousarray(q[cu[1:] - 1])          # the last position's query
     nbytes, attn_bytes = decode_bytes(lengths, hq, hk, d, masks, g)
     config = dict(bench_config(args, w, lengths, g), path="decode",
-                  l2="flush: 256 MB written before every step (the step moves %.0f MB)"
-                     % (nbytes / 1e6))
+                  l2="inputs larger than L2: the steps rotate over %d copies of the cache "
+                     "(%.0f MB; the step moves %.0f MB), no flush" % (
+                         DECODE_CACHES, DECODE_CACHES * nbytes / 1e6, nbytes / 1e6))
     if args.impl == "reference":
         if rank == 0:
             t0 = time.perf_counter()
@@ -591,11 +595,16 @@ def run_decode(args):
     dec = tm.TileMixDecode(cu[:-1], lengths, ck[:-1], cq[:-1], hq, hk, d, masks, g, int(ck[-1]),
                            device=dev)
     od = torch.empty_like(qd)
+    # Copies of the cache, used in turn: each step reads a cache the L2 has
+    # not held since DECODE_CACHES - 1 other caches were read (the decode
+    # inputs alone fit the L2).  A 256 MB write flush is measured too: it also
+    # charges the step for writing the flushed lines back.
+    caches = [(kd, vd, k8, ks)] + [(kd.clone(), vd.clone(), k8.clone(), ks.clone())
+                                   for _ in range(DECODE_CACHES - 1)]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    for _ in range(args.warmup):
-        flush.zero_()
-        dec(qd, kd, vd, k8, ks, od)
+    for it in range(args.warmup):
+        dec(qd, *caches[it % DECODE_CACHES], od)
     rc = tm.tilemix_get_error(stream)
     if rc != tm.OK:
         raise tm.TileMixError(rc, "warm-up")
@@ -613,15 +622,27 @@ def run_decode(args):
     torch.cuda.synchronize(dev)
     sampler.start()
     time.sleep(0.3)
-    for (a, b), e in zip(ev, kev):
-        flush.zero_()                     # the step's reads come from HBM, not L2
+    for it, ((a, b), e) in enumerate(zip(ev, kev)):
         a.record(stream)
-        dec(qd, kd, vd, k8, ks, od, events=e)
+        dec(qd, *caches[it % DECODE_CACHES], od, events=e)
         b.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    # the same kernel after a 256 MB write flush (for comparison)
+    n_fl = max(args.steps // 4, 3)
+    kfl = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_fl)]
+    for a, b in kfl:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    for e in kfl:
+        flush.zero_()
+        dec(qd, kd, vd, k8, ks, od, events=e)
+    torch.cuda.synchronize(dev)
+    kern_ms_flush = max_over_ranks([sum(a.elapsed_time(b) for a, b in kfl) / n_fl], device=dev)[0]
     rc = tm.tilemix_get_error(stream)
     if rc != tm.OK:
         raise tm.TileMixError(rc, "timed steps")
@@ -636,11 +657,10 @@ def run_decode(args):
     ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(n_e2e)]
     torch.cuda.synchronize(dev)
-    for a, b in ev2:
-        flush.zero_()
+    for it, (a, b) in enumerate(ev2):
         a.record(stream)
         qd.copy_(qh, non_blocking=True)
-        dec(qd, kd, vd, k8, ks, od)
+        dec(qd, *caches[it % DECODE_CACHES], od)
         oh.copy_(od, non_blocking=True)
         b.record(stream)
     torch.cuda.synchronize(dev)
@@ -660,6 +680,8 @@ def run_decode(args):
                      "kernel": "decode_attn_kernel<128>", "kernel_ms": kern_ms,
                      "peak_kind": "copy bandwidth (%s)" % pk["source"],
                      "algorithmic_bytes": attn_bytes, "step_bytes": nbytes,
+                     "kernel_ms_after_write_flush": kern_ms_flush,
+                     "frac_after_write_flush": attn_bytes / (kern_ms_flush / 1e3) / 1e9 / pk["hbm_gbs"],
                      "step_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"]},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tok/s",
                 "h2d_bytes_per_step": int(q_new.nbytes), "d2h_bytes_per_step": int(q_new.nbytes)},
