@@ -96,3 +96,17 @@ def test_mass_flops_closed_form():
     tiles = nb * (nb + 1) // 2
     assert bench.mass_flops([L], hq, d, True) == 2 * hq * tiles * 64 * 64 * 2 * d
     assert bench.mass_flops([L], hq, d, False) == 2 * hq * nb * nb * 64 * 64 * 2 * d
+
+
+def test_workload_seqs_keeps_the_first_sequences():
+    # --seqs N: the first N sequences of a configuration, with their own
+    # grouping factors (the small cases the profiler captures run)
+    import synth
+    for name in synth.WORKLOADS:
+        w, lengths, g = bench.workload(name)
+        for n in (1, 2):
+            w2, l2, g2 = bench.workload(name, seqs=n)
+            assert l2 == lengths[:n] and g2 == g[:n]
+            assert (w2["hq"], w2["hk"], w2["d"], w2["template"]) == (w["hq"], w["hk"], w["d"],
+                                                                      w["template"])
+        assert bench.workload(name, seqs=None)[1] == lengths
